@@ -1,0 +1,232 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor
+// maps, and kernel launches. All device work is in fa_fwd.cuh / fa_bwd.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kVersion = 1;
+constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [rows, d] row-major 16-bit tensor, box of 64 columns x 128 rows, 128-byte swizzle.
+bool make_tmap(CUtensorMap* map, const void* ptr, long rows, int d, int dtype) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by fa_fwd and fa_bwd. Returns FA_OK to proceed, or an error;
+// *empty is set for a valid problem with no work.
+int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0 || d < 0) return FA_ERR_INVALID;
+  if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  if (N % fa::kTile != 0) return FA_ERR_UNSUPPORTED;
+  // TMA coordinates and grid indices are 32-bit
+  if (static_cast<long long>(B) * H * N >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL, bool BF16>
+int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, void* O,
+               float* L, int BH, int N, float scale, cudaStream_t stream) {
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, BF16>;
+  // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
+  // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
+  const int smem = fa::FwdLayout<D>::kBytes > 120 * 1024 ? fa::FwdLayout<D>::kBytes : 120 * 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, static_cast<uint16_t*>(O), L, N,
+                                                 scale * 1.4426950408889634074f);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool BF16>
+int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+               const CUtensorMap& dO_map, const void* O, const void* dO, const float* L,
+               void* dQ, void* dK, void* dV, int BH, int N, float scale, void* workspace,
+               cudaStream_t stream) {
+  const long rows = static_cast<long>(BH) * N;
+  float* Dv = static_cast<float*>(workspace);
+  float* Ls = Dv + rows;
+  float* dq_acc = Ls + rows;
+  {
+    const long threads = rows * (D / 8);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), L, Dv, Ls, dq_acc,
+        rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, BF16>;
+    const size_t need = fa::BwdLayout<D>::kNeeded;
+    const size_t smem = need + 1024 <= kMaxDynSmem ? need + 1024 : kMaxDynSmem;
+    if (need > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return FA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
+    kern<<<grid, fa::kBwdThreads, smem, stream>>>(
+        q, k, v, dO_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(dK), static_cast<uint16_t*>(dV),
+        N, scale, scale * 1.4426950408889634074f, static_cast<uint32_t>(smem));
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  {
+    const long n8 = rows * D / 8;
+    const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
+    fa::fa_bwd_dq_kernel<D, BF16><<<blocks, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dQ),
+                                                             scale, n8);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+// Compile-time dispatch over (d, causal, dtype).
+template <template <int, bool, bool> class F, typename... Args>
+int dispatch(int d, int causal, int dtype, Args&&... args) {
+  const bool bf = dtype == FA_BF16;
+  if (d == 64) {
+    if (causal) return bf ? F<64, true, true>::run(args...) : F<64, true, false>::run(args...);
+    return bf ? F<64, false, true>::run(args...) : F<64, false, false>::run(args...);
+  }
+  if (causal) return bf ? F<128, true, true>::run(args...) : F<128, true, false>::run(args...);
+  return bf ? F<128, false, true>::run(args...) : F<128, false, false>::run(args...);
+}
+
+template <int D, bool C, bool B>
+struct FwdRun {
+  template <typename... A>
+  static int run(A&&... a) { return launch_fwd<D, C, B>(a...); }
+};
+template <int D, bool C, bool B>
+struct BwdRun {
+  template <typename... A>
+  static int run(A&&... a) { return launch_bwd<D, C, B>(a...); }
+};
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return kVersion; }
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID: return "FA_ERR_INVALID";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int N,
+           int d, int causal, float scale, int dtype, void* stream) {
+  bool empty;
+  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L))
+    return FA_ERR_INVALID;
+  const long rows = static_cast<long>(B) * H * N;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
+      !make_tmap(&tv, V, rows, d, dtype))
+    return FA_ERR_CUDA;
+  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, O, L, B * H, N, scale,
+                          static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B < 0 || H < 0 || N < 0 || d < 0) return static_cast<size_t>(-1);
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  if (rows == 0) return 0;
+  // D and Ls (fp32 per row), then the fp32 dQ accumulator; every part 256-aligned
+  // because rows is a multiple of 128 for every supported shape.
+  return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+           const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal,
+           float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty;
+  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!Q || !K || !V || !O || !dO || !L || !dQ || !dK || !dV || !workspace)
+    return FA_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+      !aligned16(L) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FA_ERR_INVALID;
+  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID;
+  const long rows = static_cast<long>(B) * H * N;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
+      !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype))
+    return FA_ERR_CUDA;
+  return dispatch<BwdRun>(d, causal, dtype, tq, tk, tv, tdo, O, dO, L, dQ, dK, dV, B * H, N,
+                          scale, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int fa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,406 @@
+// fa_bwd.cuh -- exact attention backward for sm_100a.
+//
+// The backward keeps no N x N matrix: the forward left only the per-row log-sum-exp
+// L, and the scores are recomputed here from Q, K and V (josueisai.com
+// "flash-attention", section "Recomputar sale mas barato que recordar"). With
+// P = exp(scale * Q K^T - L) the gradients are the standard ones:
+//
+//   dV = P^T dO,   dP = dO V^T,   D_i = sum_t dO_it O_it,   dS = P * (dP - D),
+//   dQ = scale * dS K,   dK = scale * dS^T Q.
+//
+// Three kernels:
+//   fa_bwd_pre_kernel   D = rowsum(dO * O) (fp32), Ls = L * log2(e), dQacc = 0.
+//   fa_bwd_main_kernel  one CTA per 128-key tile j of one head: K_j, V_j stay in
+//                       shared memory, the CTA walks the query tiles i that see
+//                       them, accumulates dK_j and dV_j in TMEM, and adds each
+//                       dQ_i partial into the fp32 accumulator with vector atomics.
+//   fa_bwd_dq_kernel    dQ = dtype(scale * dQacc).
+//
+// Main-kernel warp roles (320 threads):
+//   warps 0-3  compute: thread r owns key row r (TMEM lane r). P^T row from S^T and
+//              L, dS^T row from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to
+//              shared memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
+//              dK_j / dV_j epilogue.
+//   warp 4     TMA producer: K_j, V_j once; Q_i, dO_i, Ls_i, D_i into a 2-stage ring.
+//   warp 5     MMA issuer (and TMEM owner), per query tile:
+//                S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (SMEM x SMEM)
+//                dV += P^T dO_i                              (P^T from TMEM)
+//                dK += dS^T Q_i, dQ_i = dS K_j                (dS from SMEM)
+//   warps 6-9  dQ drain: thread owns query row (warp % 4) * 32 + lane; copies the
+//              dQ_i tile out of TMEM and adds it to the fp32 accumulator.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kBwdThreads = 320;
+
+template <int D>
+struct BwdLayout {
+  static constexpr uint32_t kTileBytes = kTile * D * 2;
+  static constexpr uint32_t kChunkBytes = kTile * 128;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kTileBytes;
+  static constexpr uint32_t kQ = kV + kTileBytes;       // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kTileBytes;  // 2 stages
+  static constexpr uint32_t kDS = kDO + 2 * kTileBytes; // 128 keys x 128 queries, 16-bit
+  static constexpr uint32_t kDSBytes = kTile * kTile * 2;
+  static constexpr uint32_t kL = kDS + kDSBytes;        // 2 stages x 128 fp32
+  static constexpr uint32_t kDv = kL + 2 * 512;         // 2 stages x 128 fp32
+  static constexpr uint32_t kBar = kDv + 2 * 512;
+  static constexpr int kNumBars = 16;
+  static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+  static constexpr uint32_t kAbort = kTmemSlot + 8;
+  static constexpr uint32_t kNeeded = kAbort + 8;
+  // TMEM columns
+  static constexpr uint32_t tDV = 0;
+  static constexpr uint32_t tDK = D;
+  static constexpr uint32_t tS = 2 * D;
+  static constexpr uint32_t tDP = 2 * D + 128;
+  static constexpr uint32_t tDQ = (D == 128) ? tDP : 2 * D + 256;  // d=128: dQ reuses dP^T
+};
+
+enum : int {
+  kBbKVFull = 0,
+  kBbQFull = 1,   // +stage
+  kBbQEmpty = 3,  // +stage
+  kBbSFull = 5,
+  kBbDPFull = 6,
+  kBbPFull = 7,
+  kBbDSFree = 8,
+  kBbDQFull = 9,
+  kBbDQEmpty = 10,
+  kBbDone = 11,
+};
+
+// ------------------------------------------------------------------ preprocess
+// One group of D/8 threads per row: 8 elements (16 bytes) per thread.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+    fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
+                      const float* __restrict__ L, float* __restrict__ Dv,
+                      float* __restrict__ Ls, float* __restrict__ dq_acc, long rows) {
+  constexpr int kTpr = D / 8;  // threads per row
+  const long gid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long row = gid / kTpr;
+  const int part = static_cast<int>(gid % kTpr);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 o = *reinterpret_cast<const uint4*>(O + row * D + part * 8);
+    const uint4 g = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+    const uint32_t* ow = reinterpret_cast<const uint32_t*>(&o);
+    const uint32_t* gw = reinterpret_cast<const uint32_t*>(&g);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float o0, o1, g0, g1;
+      unpack2<BF16>(ow[e], o0, o1);
+      unpack2<BF16>(gw[e], g0, g1);
+      acc = fmaf(o0, g0, acc);
+      acc = fmaf(o1, g1, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && part == 0) {
+    Dv[row] = acc;
+    Ls[row] = L[row] * 1.4426950408889634074f;
+  }
+}
+
+// ------------------------------------------------------------------ dQ convert
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256)
+    fa_bwd_dq_kernel(const float* __restrict__ dq_acc, uint16_t* __restrict__ dQ, float scale,
+                     long n8) {
+  const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(dq_acc)[2 * i + 1];
+  uint4 out;
+  out.x = pack2<BF16>(a.x * scale, a.y * scale);
+  out.y = pack2<BF16>(a.z * scale, a.w * scale);
+  out.z = pack2<BF16>(b.x * scale, b.y * scale);
+  out.w = pack2<BF16>(b.z * scale, b.w * scale);
+  reinterpret_cast<uint4*>(dQ)[i] = out;
+}
+
+// --------------------------------------------------------------- main dK/dV
+template <int D, bool CAUSAL, bool BF16>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ Ls,
+                       const float* __restrict__ Dv, float* __restrict__ dq_acc,
+                       uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int N,
+                       float scale, float scale_log2, uint32_t smem_alloc) {
+  using Lay = BwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
+  if (pad + Lay::kNeeded > smem_alloc) {
+    // Shared memory is not placed as this kernel needs; report and do nothing.
+    if (threadIdx.x == 0) atomicExch(&g_fa_status, -3);
+    return;
+  }
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_base + pad;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = N / kTile;
+  const int bh = blockIdx.x / ntiles;
+  const int j = blockIdx.x - bh * ntiles;  // key tile (j = 0 has the most causal work)
+  const int i_begin = CAUSAL ? j : 0;
+  const int niter = ntiles - i_begin;
+  const long head_row = static_cast<long>(bh) * N;
+
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBbKVFull), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBbQFull + s), 1);
+      mbar_init(bar(kBbQEmpty + s), 1);
+    }
+    mbar_init(bar(kBbSFull), 1);
+    mbar_init(bar(kBbDPFull), 1);
+    mbar_init(bar(kBbPFull), 128);
+    mbar_init(bar(kBbDSFree), 1);
+    mbar_init(bar(kBbDQFull), 1);
+    mbar_init(bar(kBbDQEmpty), 128);
+    mbar_init(bar(kBbDone), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + Lay::kTmemSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch(&tmQ);
+      tma_prefetch(&tmK);
+      tma_prefetch(&tmV);
+      tma_prefetch(&tmDO);
+      const int krow = static_cast<int>(head_row) + j * kTile;
+      mbar_expect_tx(bar(kBbKVFull), 2 * Lay::kTileBytes);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_2d(sbase + Lay::kK + c * Lay::kChunkBytes, &tmK, c * 64, krow, bar(kBbKVFull));
+        tma_load_2d(sbase + Lay::kV + c * Lay::kChunkBytes, &tmV, c * 64, krow, bar(kBbKVFull));
+      }
+      for (int it = 0; it < niter; ++it) {
+        const int st = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (it >= 2 && !mbar_wait(bar(kBbQEmpty + st), (use - 1) & 1, abort_flag)) break;
+        const int qrow = static_cast<int>(head_row) + (i_begin + it) * kTile;
+        const uint32_t full = bar(kBbQFull + st);
+        mbar_expect_tx(full, 2 * Lay::kTileBytes + 2 * 512);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
+                      qrow, full);
+          tma_load_2d(sbase + Lay::kDO + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmDO,
+                      c * 64, qrow, full);
+        }
+        bulk_load(sbase + Lay::kL + st * 512, Ls + qrow, 512, full);
+        bulk_load(sbase + Lay::kDv + st * 512, Dv + qrow, 512, full);
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_sq = idesc_f16_f32(kTile, kTile, BF16, false, false);  // S^T, dP^T
+      constexpr uint32_t id_acc = idesc_f16_f32(kTile, D, BF16, false, true);      // dV, dK
+      constexpr uint32_t id_dq = idesc_f16_f32(kTile, D, BF16, true, true);        // dQ
+      const uint32_t sk = sbase + Lay::kK, sv = sbase + Lay::kV, sds = sbase + Lay::kDS;
+      bool ok = mbar_wait(bar(kBbKVFull), 0, abort_flag);
+      for (int it = 0; ok && it < niter; ++it) {
+        const int st = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        const uint32_t ph = static_cast<uint32_t>(it & 1);
+        const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
+        const uint32_t sdo = sbase + Lay::kDO + st * Lay::kTileBytes;
+        if (!mbar_wait(bar(kBbQFull + st), use & 1, abort_flag)) break;
+        tc_fence_after();
+        // S^T = K_j Q_i^T
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tS, sdesc_sw128(sk + off, 16, 1024), sdesc_sw128(sq + off, 16, 1024),
+                 id_sq, k > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBbSFull));
+        // dP^T = V_j dO_i^T, into columns the previous dQ tile may still occupy
+        if (it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tDP, sdesc_sw128(sv + off, 16, 1024),
+                 sdesc_sw128(sdo + off, 16, 1024), id_sq, k > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(kBbDPFull));
+        if (!mbar_wait(bar(kBbPFull), ph, abort_flag)) break;
+        tc_fence_after();
+        // dV += P^T dO_i  (K = the 128 queries of tile i)
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k)
+          mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8,
+                 sdesc_sw128(sdo + k * 2048, Lay::kChunkBytes, 1024), id_acc,
+                 (it > 0 || k > 0) ? 1u : 0u);
+        // dK += dS^T Q_i
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k) {
+          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tDK, sdesc_sw128(sds + off, 16, 1024),
+                 sdesc_sw128(sq + k * 2048, Lay::kChunkBytes, 1024), id_acc,
+                 (it > 0 || k > 0) ? 1u : 0u);
+        }
+        // dQ_i = dS K_j   (dS read M-major from the same shared tile)
+#pragma unroll
+        for (int k = 0; k < kTile / 16; ++k)
+          mma_ss(tmem + Lay::tDQ, sdesc_sw128(sds + k * 2048, Lay::kChunkBytes, 1024),
+                 sdesc_sw128(sk + k * 2048, Lay::kChunkBytes, 1024), id_dq, k > 0 ? 1u : 0u);
+        mma_commit(bar(kBbQEmpty + st));
+        mma_commit(bar(kBbDSFree));
+        mma_commit(bar(kBbDQFull));
+      }
+      mma_commit(bar(kBbDone));
+    }
+  } else if (warp < 4) {
+    // ----------------------------------------------------------------- compute
+    const int r = warp * 32 + lane;  // key row within the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    uint8_t* sds_row = smem + Lay::kDS + r * 128;
+    const int sw = r & 7;
+    bool ok = true;
+    for (int it = 0; it < niter; ++it) {
+      const int st = it & 1;
+      const uint32_t ph = static_cast<uint32_t>(it & 1);
+      const bool diag = CAUSAL && (i_begin + it == j);
+      if (!mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) ||
+          !mbar_wait(bar(kBbSFull), ph, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const float* sL = reinterpret_cast<const float*>(smem + Lay::kL + st * 512);
+      const float* sD = reinterpret_cast<const float*>(smem + Lay::kDv + st * 512);
+      float p[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(lane_base + Lay::tS + c * 32, sr);
+        tmem_wait_ld();
+        reg_fence32(sr);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int q = c * 32 + e;
+          float x = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, -sL[q]));
+          if (diag && q < r) x = 0.f;
+          p[q] = x;
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(p[c * 32 + 2 * e], p[c * 32 + 2 * e + 1]);
+        tmem_st16(lane_base + Lay::tS + c * 16, pk);
+      }
+      if (!mbar_wait(bar(kBbDPFull), ph, abort_flag)) { ok = false; break; }
+      if (it > 0 && !mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) {
+        uint32_t dr[32];
+        tmem_ld32(lane_base + Lay::tDP + c * 32, dr);
+        tmem_wait_ld();
+        reg_fence32(dr);
+        uint32_t ds[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int q = c * 32 + 2 * e;
+          const float a = p[q] * (__uint_as_float(dr[2 * e]) - sD[q]);
+          const float b = p[q + 1] * (__uint_as_float(dr[2 * e + 1]) - sD[q + 1]);
+          ds[e] = pack2<BF16>(a, b);
+        }
+        // queries c*32 .. c*32+31 = 16-byte units u0..u0+3 of swizzle column c/2
+        uint8_t* base = sds_row + (c >> 1) * Lay::kChunkBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int unit = ((c & 1) * 4 + u) ^ sw;
+          *reinterpret_cast<uint4*>(base + unit * 16) =
+              make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
+        }
+      }
+      fence_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBbPFull));
+    }
+    if (ok && mbar_wait(bar(kBbDone), 0, abort_flag)) {
+      tc_fence_after();
+      const long grow = head_row + static_cast<long>(j) * kTile + r;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? Lay::tDV : Lay::tDK;
+        const float mul = which == 0 ? 1.f : scale;
+        uint16_t* dst_row = (which == 0 ? dV : dK) + grow * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + col + c * 32, v);
+          tmem_wait_ld();
+          reg_fence32(v);
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pw[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+        }
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- dQ drain
+    const int quarter = warp & 3;
+    const int qr = quarter * 32 + lane;  // query row within tile i
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    for (int it = 0; it < niter; ++it) {
+      if (!mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)) break;
+      tc_fence_after();
+      uint32_t v[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
+      tc_fence_before();
+      mbar_arrive(bar(kBbDQEmpty));
+      float4* dst = reinterpret_cast<float4*>(
+          dq_acc + (head_row + static_cast<long>(i_begin + it) * kTile + qr) * D);
+#pragma unroll
+      for (int e = 0; e < D / 4; ++e)
+        atomicAdd(dst + e, make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,274 @@
+// fa_fwd.cuh -- exact attention forward for sm_100a.
+//
+// One CTA owns one 128-row query tile of one (batch, head) and walks the key/value
+// tiles of that head, block by block, with the online softmax of josueisai.com
+// "flash-attention", section "El truco: trocear y llevar la cuenta del softmax":
+// per row a running maximum m and running sum l; when m grows the partial output is
+// rescaled, and after the last block the output is divided by l once. The N x N
+// score and probability tiles live only in tensor memory (TMEM); Q, K, V are read
+// from HBM once per CTA ("una pasada sobre Q, K y V", same page, comparison table).
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Loads its score row
+//              from TMEM, masks, updates m and l, writes P (16-bit) back into TMEM
+//              over the scores, rescales its O row when m grew, and runs the epilogue.
+//   warp 4     TMA producer: Q once, then K_j / V_j into a 2-stage ring.
+//   warp 5     MMA issuer: S_j = Q K_j^T (SMEM x SMEM -> TMEM, fp32) and
+//              O += P_j V_j (P from TMEM, V from SMEM -> TMEM, fp32). It also owns
+//              the TMEM allocation.
+//
+// TMEM (512 columns x 128 lanes of 32 bit): S/P buffer 0 at column 0, S/P buffer 1
+// at column 128, O at column 256 (d columns). S_{j+1} is computed while the softmax
+// warps work on S_j.
+//
+// Scores are kept in the base-2 domain: s' = s * scale * log2(e), p = 2^(s' - m').
+// The running reference m' is only moved when the row maximum exceeds it by more
+// than kRescaleSlack (so exponentials stay <= 2^kRescaleSlack); the result is the
+// same because l, O and L all share whatever reference is current.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr int kFwdThreads = 192;
+constexpr float kRescaleSlack = 8.0f;
+
+template <int D>
+struct FwdLayout {
+  static constexpr uint32_t kTileBytes = kTile * D * 2;  // 128 rows x D 16-bit values
+  static constexpr uint32_t kChunkBytes = kTile * 128;   // 128 rows x 64 values (one swizzle column)
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + kTileBytes;        // 2 stages
+  static constexpr uint32_t kV = kK + 2 * kTileBytes;    // 2 stages
+  static constexpr uint32_t kBar = kV + 2 * kTileBytes;
+  static constexpr int kNumBars = 12;
+  static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+  static constexpr uint32_t kAbort = kTmemSlot + 8;
+  static constexpr uint32_t kBytes = kAbort + 8 + 1024;  // + alignment slack
+};
+
+// barrier indices
+enum : int {
+  kBarQFull = 0,
+  kBarKFull = 1,   // +stage
+  kBarVFull = 3,   // +stage
+  kBarKVEmpty = 5, // +stage
+  kBarSFull = 7,   // +buffer
+  kBarPFull = 9,   // +buffer
+  kBarODone = 11,
+};
+
+template <int D, bool CAUSAL, bool BF16>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, uint16_t* __restrict__ O,
+                  float* __restrict__ Lse, int N, float scale_log2) {
+  using Lay = FwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_base + pad;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = N / kTile;
+  const int bh = blockIdx.x / ntiles;
+  const int tr = blockIdx.x - bh * ntiles;
+  const int t = CAUSAL ? (ntiles - 1 - tr) : tr;  // heaviest causal tiles first
+  const int nkv = CAUSAL ? t + 1 : ntiles;
+  const int row0 = bh * N + t * kTile;              // first row in the [B*H*N, D] view
+
+  auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQFull), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarKVEmpty + s), 1);
+      mbar_init(bar(kBarSFull + s), 1);
+      mbar_init(bar(kBarPFull + s), 128);
+    }
+    mbar_init(bar(kBarODone), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + Lay::kTmemSlot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch(&tmQ);
+      tma_prefetch(&tmK);
+      tma_prefetch(&tmV);
+      mbar_expect_tx(bar(kBarQFull), Lay::kTileBytes);
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_2d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, row0, bar(kBarQFull));
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j & 1;
+        const uint32_t use = static_cast<uint32_t>(j >> 1);
+        if (j >= 2 && !mbar_wait(bar(kBarKVEmpty + st), (use - 1) & 1, abort_flag)) break;
+        const int krow = bh * N + j * kTile;
+        const uint32_t sk = sbase + Lay::kK + st * Lay::kTileBytes;
+        const uint32_t sv = sbase + Lay::kV + st * Lay::kTileBytes;
+        mbar_expect_tx(bar(kBarKFull + st), Lay::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sk + c * Lay::kChunkBytes, &tmK, c * 64, krow, bar(kBarKFull + st));
+        mbar_expect_tx(bar(kBarVFull + st), Lay::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sv + c * Lay::kChunkBytes, &tmV, c * 64, krow, bar(kBarVFull + st));
+      }
+    }
+  } else if (warp == 5) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_f16_f32(kTile, kTile, BF16, false, false);
+      constexpr uint32_t idesc_o = idesc_f16_f32(kTile, D, BF16, false, true);
+      const uint32_t sq = sbase + Lay::kQ;
+      bool ok = mbar_wait(bar(kBarQFull), 0, abort_flag);
+      for (int j = 0; ok && j <= nkv; ++j) {
+        if (j < nkv) {
+          const int st = j & 1;
+          const uint32_t use = static_cast<uint32_t>(j >> 1);
+          if (!mbar_wait(bar(kBarKFull + st), use & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t sk = sbase + Lay::kK + st * Lay::kTileBytes;
+          const uint32_t d_s = tmem + st * 128;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+            mma_ss(d_s, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc_s,
+                   k > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(kBarSFull + st));
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int b = jj & 1;
+          const uint32_t use = static_cast<uint32_t>(jj >> 1);
+          if (!mbar_wait(bar(kBarPFull + b), use & 1, abort_flag)) break;
+          if (!mbar_wait(bar(kBarVFull + b), use & 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t sv = sbase + Lay::kV + b * Lay::kTileBytes;
+          const uint32_t a_p = tmem + b * 128;  // P packed in the first 64 columns
+          const uint32_t d_o = tmem + 256;
+#pragma unroll
+          for (int k = 0; k < kTile / 16; ++k) {
+            mma_ts(d_o, a_p + k * 8, sdesc_sw128(sv + k * 2048, Lay::kChunkBytes, 1024), idesc_o,
+                   (jj > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(kBarKVEmpty + b));
+          mma_commit(bar(kBarODone));
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------- softmax
+    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float m = -INFINITY;  // running reference, base-2 scaled units
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int b = j & 1;
+      const uint32_t use = static_cast<uint32_t>(j >> 1);
+      if (!mbar_wait(bar(kBarSFull + b), use & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) tmem_ld32(lane_base + b * 128 + c * 32, sr + c * 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < kTile / 32; ++c) reg_fence32(sr + c * 32);
+      float s[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sr[c]);
+      if (CAUSAL && j == t) {
+#pragma unroll
+        for (int c = 0; c < kTile; ++c)
+          if (c > r) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, s[c]);
+      const float cand = mx * scale_log2;
+      const float m_new = (cand > m + kRescaleSlack) ? cand : m;
+      const float alpha = ex2_approx(m - m_new);  // 0 on the first tile, 1 if unchanged
+      float rowsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const float p = ex2_approx(fmaf(s[c], scale_log2, -m_new));
+        rowsum += p;
+        s[c] = p;
+      }
+      l = l * alpha + rowsum;
+      uint32_t pk[kTile / 2];
+#pragma unroll
+      for (int c = 0; c < kTile / 2; ++c) pk[c] = pack2<BF16>(s[2 * c], s[2 * c + 1]);
+      tmem_st32(lane_base + b * 128, pk);
+      tmem_st32(lane_base + b * 128 + 32, pk + 32);
+      if (j > 0) {
+        // the previous P V must have landed before O is touched
+        if (!mbar_wait(bar(kBarODone), (j - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + 256 + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_base + 256 + c * 32, o);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + b));
+      m = m_new;
+    }
+    if (ok && mbar_wait(bar(kBarODone), (nkv - 1) & 1, abort_flag)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      uint16_t* orow = O + static_cast<size_t>(row0 + r) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + 256 + c * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        uint4 pkd[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pw[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = pkd[e];
+      }
+      Lse[row0 + r] = (m + log2f(l)) * 0.69314718055994530942f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,147 @@
+"""ctypes binding of libfa.so (include/fa.h): argument marshalling only.
+
+Every step of the attention computation runs in the library's CUDA kernels; this
+module turns torch tensors into device pointers and the current CUDA stream, and
+turns status codes into exceptions. It never computes attention itself, and it
+raises if the library is missing -- there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK = 0
+FA_ERR_INVALID = -1
+FA_ERR_UNSUPPORTED = -2
+FA_ERR_CUDA = -3
+FA_ERR_TIMEOUT = -4
+FA_BF16 = 0
+FA_FP16 = 1
+
+# Every symbol include/fa.h declares, with its ctypes signature.
+_vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32, _int, _vp]),
+    "fa_bwd_workspace_size": (_sz, [_int, _int, _int, _int]),
+    "fa_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int,
+                      _f32, _int, _vp, _sz, _vp]),
+    "fa_get_device_status": (_int, [_vp]),
+    "fa_status_string": (ctypes.c_char_p, [_int]),
+    "fa_version": (_int, []),
+}
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def load():
+    """Load libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m exact_io_aware_69_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    raise FaError(FA_ERR_UNSUPPORTED, f"dtype {t.dtype}")
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, like=None):
+    if not t.is_cuda:
+        raise FaError(FA_ERR_INVALID, f"{name} is not a CUDA tensor")
+    if not t.is_contiguous():
+        raise FaError(FA_ERR_INVALID, f"{name} is not contiguous")
+    if like is not None and (t.shape != like.shape or t.dtype != like.dtype):
+        raise FaError(FA_ERR_INVALID, f"{name} shape/dtype differs from q")
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+            stream=None):
+    """O, L = attention(q, k, v) for [B, H, N, d] bf16/fp16 CUDA tensors."""
+    import torch
+    lib = load()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, q)
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                    B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
+                    _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+    return out, lse
+
+
+def workspace_size(B, H, N, d) -> int:
+    return int(load().fa_bwd_workspace_size(B, H, N, d))
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
+             workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV of attention, recomputing P from q, k, v and the forward's lse."""
+    import torch
+    lib = load()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _check(t, n, q)
+    _check(lse, "lse")
+    B, H, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+                    int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
+                    workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error word."""
+    return int(load().fa_get_device_status(_stream_handle(stream)))

@@ -1,0 +1,110 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library, libfa.so.
+ *
+ * Operation. Exact scaled-dot-product attention, per batch b and head h:
+ *
+ *   S = scale * Q K^T          (N x N, never stored)
+ *   P = softmax(S) by rows     (N x N, never stored)
+ *   O = P V
+ *
+ * the three steps of josueisai.com "flash-attention", section "La matriz que nunca
+ * deberias guardar", computed tile by tile with the online softmax of section "El
+ * truco: trocear y llevar la cuenta del softmax" so that S and P stay on chip. The
+ * forward also writes the per-row log-sum-exp L (kerneldigest.dev "FlashAttention",
+ * first paragraph: online log-sum-exp scaling). The backward keeps no P: it
+ * recomputes the scores from Q, K, V and uses L (josueisai.com, section "Recomputar
+ * sale mas barato que recordar").
+ *
+ * Causal mask (optional; not on the pages): key j is visible to query i iff j <= i,
+ * top-left aligned, N_q = N_k = N.
+ *
+ * Layout. Every 16-bit tensor (Q, K, V, O, dO, dQ, dK, dV) is a dense row-major
+ * [B][H][N][d] array of one element type (bf16 or fp16, the `dtype` argument), so
+ * element (b, h, n, t) sits at ((b*H + h)*N + n)*d + t. L is fp32 [B][H][N], in
+ * natural-log units of the scaled score: L_i = m_i + ln(sum_j exp(s_ij - m_i)).
+ * Arithmetic is fp32 with 16-bit MMA operands (P and dS are rounded to `dtype`
+ * before their products).
+ *
+ * Pointers are DEVICE pointers and must be 16-byte aligned. `stream` is a
+ * cudaStream_t (NULL = legacy default stream). Every call only enqueues work on
+ * `stream` and returns; outputs are valid once the stream has reached that point.
+ *
+ * Ownership. The caller allocates and owns every buffer, including the backward
+ * workspace sized by fa_bwd_workspace_size(). The library allocates no device
+ * memory in these calls; its only state is one device-side error word per device.
+ *
+ * Supported now: d in {64, 128}; N a positive multiple of 128; dtype bf16 or fp16.
+ *
+ * Errors are checked on the host before anything is enqueued and are returned as
+ * codes (no exception, no abort, no fallback to another implementation):
+ *   FA_ERR_INVALID      null pointer, negative size, misaligned pointer, a workspace
+ *                       that is too small, or a non-finite / non-positive scale;
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, N % 128 != 0;
+ *   FA_ERR_CUDA         a CUDA runtime/driver call or a launch failed;
+ *   FA_ERR_TIMEOUT      (from fa_get_device_status only) a kernel gave up a bounded
+ *                       wait on the device and returned without finishing.
+ * B*H*N == 0 is a valid empty problem: FA_OK, nothing is enqueued.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID = -1,
+    FA_ERR_UNSUPPORTED = -2,
+    FA_ERR_CUDA = -3,
+    FA_ERR_TIMEOUT = -4
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward. Reads Q, K, V [B][H][N][d]; writes O [B][H][N][d] (dtype) and
+ * L [B][H][N] (fp32). One kernel launch.
+ */
+int fa_fwd(const void *Q, const void *K, const void *V, void *O, float *L, int B, int H, int N,
+           int d, int causal, float scale, int dtype, void *stream);
+
+/*
+ * Bytes of device workspace that fa_bwd needs for this shape: fp32 D and scaled L
+ * ([B][H][N] each) plus an fp32 dQ accumulator [B][H][N][d]. 0 for an empty
+ * problem; (size_t)-1 for sizes that fa_bwd rejects as invalid.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward. Given Q, K, V, the forward's O and L, and dO, writes dQ, dK, dV
+ * ([B][H][N][d], dtype). `workspace` is a caller-owned device buffer of at least
+ * fa_bwd_workspace_size(B, H, N, d) bytes, 256-byte aligned; its contents on entry
+ * do not matter and on return are scratch. Four kernel launches: D = rowsum(dO * O)
+ * and zeroing of the dQ accumulator; the dK/dV pass that recomputes P from L and
+ * adds dQ partials atomically; the conversion of dQ to dtype.
+ */
+int fa_bwd(const void *Q, const void *K, const void *V, const void *O, const void *dO,
+           const float *L, void *dQ, void *dK, void *dV, int B, int H, int N, int d, int causal,
+           float scale, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device error word of the
+ * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel abandoned a bounded wait.
+ * FA_ERR_CUDA if the synchronisation itself failed.
+ */
+int fa_get_device_status(void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *fa_status_string(int status);
+
+/* Library version, for the binding's load check. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI (no GPU needed, nothing is launched).
+
+The library must load on a machine without a GPU, export every function that
+include/fa.h declares, and reject bad arguments with the documented status code
+before touching the device.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_69_b200 import build, fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return fa.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    assert names == sorted(["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_status",
+                            "fa_status_string", "fa_version"])
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert name in fa.SIGNATURES, name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.fa_version() == 1
+    for code, text in [(0, "FA_OK"), (-1, "FA_ERR_INVALID"), (-2, "FA_ERR_UNSUPPORTED"),
+                       (-3, "FA_ERR_CUDA"), (-4, "FA_ERR_TIMEOUT"), (7, "FA_ERR_UNKNOWN")]:
+        assert fa.status_string(code) == text
+
+
+def test_workspace_size(lib):
+    assert lib.fa_bwd_workspace_size(2, 3, 256, 64) == 2 * 3 * 256 * (8 + 64 * 4)
+    assert lib.fa_bwd_workspace_size(0, 3, 256, 64) == 0
+    assert lib.fa_bwd_workspace_size(-1, 3, 256, 64) == ctypes.c_size_t(-1).value
+
+
+# Fake, well-aligned device addresses: validation must reject before any use.
+P = 0x7F0000000000
+
+
+def _fwd(lib, **kw):
+    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, L=P + 0x400000, B=1, H=1,
+             N=256, d=64, causal=0, scale=0.125, dtype=fa.FA_BF16, stream=None)
+    a.update(kw)
+    return lib.fa_fwd(a["Q"], a["K"], a["V"], a["O"], a["L"], a["B"], a["H"], a["N"], a["d"],
+                      a["causal"], a["scale"], a["dtype"], a["stream"])
+
+
+def _bwd(lib, **kw):
+    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, dO=P + 0x400000,
+             L=P + 0x500000, dQ=P + 0x600000, dK=P + 0x700000, dV=P + 0x800000, B=1, H=1, N=256,
+             d=64, causal=0, scale=0.125, dtype=fa.FA_BF16, ws=P + 0x900000, ws_bytes=1 << 30,
+             stream=None)
+    a.update(kw)
+    return lib.fa_bwd(a["Q"], a["K"], a["V"], a["O"], a["dO"], a["L"], a["dQ"], a["dK"], a["dV"],
+                      a["B"], a["H"], a["N"], a["d"], a["causal"], a["scale"], a["dtype"], a["ws"],
+                      a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), fa.FA_ERR_INVALID),
+    (dict(L=None), fa.FA_ERR_INVALID),
+    (dict(B=-1), fa.FA_ERR_INVALID),
+    (dict(N=-128), fa.FA_ERR_INVALID),
+    (dict(K=P + 8), fa.FA_ERR_INVALID),
+    (dict(scale=0.0), fa.FA_ERR_INVALID),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(N=200), fa.FA_ERR_UNSUPPORTED),
+    (dict(dtype=2), fa.FA_ERR_UNSUPPORTED),
+    (dict(B=0), fa.FA_OK),
+    (dict(N=0, Q=None, K=None, V=None, O=None, L=None), fa.FA_OK),
+])
+def test_fwd_rejects_before_launch(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dO=None), fa.FA_ERR_INVALID),
+    (dict(ws=None), fa.FA_ERR_INVALID),
+    (dict(ws=P + 0x900010), fa.FA_ERR_INVALID),  # workspace must be 256-byte aligned
+    (dict(ws_bytes=1000), fa.FA_ERR_INVALID),
+    (dict(dV=P + 0x800002), fa.FA_ERR_INVALID),
+    (dict(H=-2), fa.FA_ERR_INVALID),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(N=130), fa.FA_ERR_UNSUPPORTED),
+    (dict(dtype=5), fa.FA_ERR_UNSUPPORTED),
+    (dict(H=0), fa.FA_OK),
+])
+def test_bwd_rejects_before_launch(lib, kw, code):
+    assert _bwd(lib, **kw) == code
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(fa, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(fa, "_lib", None)
+    with pytest.raises(ImportError):
+        fa.load()
