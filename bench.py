@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Throughput of exact attention forward + backward on B200, through the C ABI.
+
+One step = one pass of the whole hot path over one batch: the forward kernel
+(O, L) and the three backward kernels (preprocess, dK/dV with atomic dQ, dQ
+conversion) on the workload B=2, H=32, N=8192, d=128, bf16, causal (the ~8k-token
+case of 64 M scores per head). Inputs are seeded synthetic iid N(0,1) values already
+resident in HBM when the timed region starts; Q, K, V, dO are 134 MB each, larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0. --impl reference times the fp64 CPU oracle on a
+bounded sample of the same workload instead (the oracle is the only reference this
+method has).
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run (one process per GPU, each an independent replica: the
+attention problems are independent, so there is no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from exact_io_aware_69_b200.inputs import WORKLOADS  # noqa: E402
+
+METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16, causal/non) and % of tensor-core peak"
+UNIT = "TFLOP/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c3", choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def flops(w):
+    """(fwd, bwd) algorithmic FLOPs: fwd 4*B*H*N^2*d (halved for causal), bwd 2.5 x fwd."""
+    f = w.fwd_flops()
+    return f, 2.5 * f
+
+
+def config_of(w):
+    return {
+        "workload": f"B{w.B} H{w.H} N{w.N} d{w.d} {w.dtype} {'causal' if w.causal else 'non-causal'}"
+                    " exact attention fwd+bwd",
+        "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "scale": "1/sqrt(d)",
+        "l2": "inputs larger than L2 (Q, K, V, dO %.0f MB each > 126 MB), no flush"
+              % (w.B * w.H * w.N * w.d * 2 / 1e6),
+        "flop_convention": "fwd = 4*B*H*N^2*d, halved for causal; value = fwd+bwd counted as "
+                           "2.5 x fwd as the target states; 'fwd_bwd_tflops_3p5x' counts the "
+                           "five backward GEMMs too (3.5 x fwd)",
+        "parallelism": "replicas (one independent problem per GPU)",
+    }
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_69_b200", "csrc", "*"))):
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this source."""
+    try:
+        with open(TRAFFIC_FILE) as fh:
+            t = json.load(fh)
+    except OSError:
+        return None
+    e = t.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash() or e.get("workload") != workload:
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.out = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+        self.sel = []
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.fh = open(self.out, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.out) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.out)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # samples under load: the top part of the distribution (idle edges excluded)
+        hi = [s for s in sm if s >= 0.5 * max(sm)]
+        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def run_reference(args, w, rank):
+    """The oracle as it stands, timed on this host's cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    inp = w.make()
+    d = w.d
+    BH = w.B * w.H
+    sample_heads = [0]
+    qf, kf, vf, df = (inp.widened(n).reshape(BH, w.N, d)[sample_heads].astype(np.float64)
+                      for n in ("q", "k", "v", "do"))
+    fwd_f, bwd_f = flops(w)
+    step_flops = 2.5 * fwd_f / BH * len(sample_heads)
+    for _ in range(args.warmup):
+        oracle.attn_bwd(qf, kf, vf, df, w.causal, w.scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attn_bwd(qf, kf, vf, df, w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    value = step_flops * args.steps / dt / 1e12
+    cores = oracle.num_threads()
+    sample = f"head 0 of {BH} (fwd+bwd, all {w.N} rows) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded iid N(0,1), rounded to bf16)", "config": config_of(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_and_parity(w, inp, outs, target_s):
+    """Time the oracle on whole heads until ~target_s of CPU work; check the GPU's
+    outputs for those heads against it."""
+    import oracle
+    BH, N, d = w.B * w.H, w.N, w.d
+    fwd_f, bwd_f = flops(w)
+    per_head = 2.5 * fwd_f / BH
+    q, k, v, do = (inp.widened(n).reshape(BH, N, d) for n in ("q", "k", "v", "do"))
+    heads, elapsed = [], 0.0
+    worst = {}
+    order = [0, BH - 1] + list(range(1, BH - 1))
+    while elapsed < target_s and len(heads) < BH:
+        h = order[len(heads)]
+        args = [x[h:h + 1].astype(np.float64) for x in (q, k, v, do)]
+        t0 = time.perf_counter()
+        ref = oracle.attn_bwd(*args, w.causal, w.scale)
+        elapsed += time.perf_counter() - t0
+        heads.append(h)
+        for name in ("o", "dq", "dk", "dv"):
+            got = outs[name].reshape(BH, N, d)[h].astype(np.float64)
+            diff = np.abs(got - ref[name][0])
+            rel = float((diff / np.maximum(1.0, np.abs(ref[name][0]))).max())
+            cur = worst.get(name, (0.0, 0.0))
+            worst[name] = (max(cur[0], rel), max(cur[1], float(diff.mean())))
+        dl = float(np.abs(outs["L"].reshape(BH, N)[h] - ref["L"][0]).max())
+        worst["L"] = (max(worst.get("L", (0.0, 0.0))[0], dl), 0.0)
+    tol_max, tol_mean = (2e-2, 2e-3) if w.dtype == "bf16" else (5e-3, 5e-4)
+    ok = all(worst[n][0] <= tol_max and worst[n][1] <= tol_mean for n in ("o", "dq", "dk", "dv"))
+    ok = ok and worst["L"][0] <= 1e-3
+    base = {"value": per_head * len(heads) / elapsed / 1e12, "unit": UNIT,
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(heads)} of {BH} heads (fwd+bwd, all {N} rows each), "
+                      f"{elapsed:.1f} s of fp64 CPU work"}
+    parity = {"heads_checked": heads, "ok": bool(ok),
+              "max_err": {n: round(worst[n][0], 6) for n in worst},
+              "mean_abs_err": {n: round(worst[n][1], 7) for n in ("o", "dq", "dk", "dv")},
+              "reading": "max |got-ref|/max(1,|ref|) vs 2e-2, mean |got-ref| vs 2e-3, L abs 1e-3"}
+    return base, parity
+
+
+def main():
+    args = parse_args()
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+
+    import torch
+    from exact_io_aware_69_b200 import fa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=dev)
+        pg = dist
+
+    fa.load()
+    stream = torch.cuda.current_stream()
+    B, H, N, d = w.B, w.H, w.N, w.d
+    inp = w.make()
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+
+    def pinned(bits):
+        t = torch.from_numpy(bits.view(np.int16)).view(tdt)
+        return t.pin_memory()
+
+    h_in = {n: pinned(getattr(inp, n)) for n in ("q", "k", "v", "do")}
+    dv_in = {n: t.to(dev) for n, t in h_in.items()}
+    q, k, v, do = dv_in["q"], dv_in["k"], dv_in["v"], dv_in["do"]
+    o = torch.empty_like(q)
+    L = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dvv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
+    scale = w.scale
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        fa.backward_stage("preprocess", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        fa.backward_stage("dkdv", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        fa.backward_stage("dq_convert", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.device_status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(events[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per_kernel = {"fa_fwd_kernel": 0.0, "fa_bwd_pre_kernel": 0.0, "fa_bwd_main_kernel": 0.0,
+                  "fa_bwd_dq_kernel": 0.0}
+    names = list(per_kernel)
+    for ev in events:
+        for i, n in enumerate(names):
+            per_kernel[n] += ev[i].elapsed_time(ev[i + 1])
+    if pg:
+        t = torch.tensor([total_ms] + [per_kernel[n] for n in names], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t[0])
+        for i, n in enumerate(names):
+            per_kernel[n] = float(t[1 + i])
+    st = fa.device_status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status {st} after timing")
+
+    fwd_f, bwd_f = flops(w)
+    steps = args.steps
+    ms_step = total_ms / steps
+    # fwd+bwd counted as 2.5 x fwd, literally as the target states it
+    value = world * (2.5 * fwd_f) * steps / (total_ms * 1e-3) / 1e12
+    fwd_ms = per_kernel["fa_fwd_kernel"] / steps
+    bwd_ms = sum(per_kernel[n] for n in names[1:]) / steps
+    peaks, peak_kind = load_peaks()
+    peak_burst = float(peaks["bf16_tflops"])
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak_burst))
+
+    # dominant kernel: the largest share of the step
+    kflops = {"fa_fwd_kernel": fwd_f, "fa_bwd_main_kernel": bwd_f}
+    rows = B * H * N
+    kbytes = {"fa_bwd_pre_kernel": rows * d * 2 * 2 + rows * 4 + rows * 8 + rows * d * 4,
+              "fa_bwd_dq_kernel": rows * d * 4 + rows * d * 2}
+    dom = max(per_kernel, key=per_kernel.get)
+    dom_ms = per_kernel[dom] / steps
+    if dom in kflops:
+        achieved = kflops[dom] / (dom_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
+                "unit": "TFLOP/s", "frac": achieved / peak_sus,
+                "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside the step loop)",
+                "frac_of_burst_peak": achieved / peak_burst,
+                "algorithmic_per_launch": kflops[dom], "avg_launch_ms": dom_ms}
+    else:
+        achieved = kbytes[dom] / (dom_ms * 1e-3) / 1e9
+        hbm = float(peaks["hbm_gbs"])
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_kind": f"{peak_kind} HBM copy",
+                "algorithmic_per_launch": kbytes[dom], "avg_launch_ms": dom_ms}
+    roof["traffic"] = recorded_traffic(dom, args.workload)
+
+    kernels = {}
+    for n in names:
+        ms = per_kernel[n] / steps
+        e = {"avg_ms": ms, "share": per_kernel[n] / sum(per_kernel.values())}
+        if n in kflops:
+            e["tflops"] = kflops[n] / (ms * 1e-3) / 1e12
+            e["frac_of_sustained_peak"] = e["tflops"] / peak_sus
+        else:
+            e["gbs"] = kbytes[n] / (ms * 1e-3) / 1e9
+        kernels[n] = e
+
+    # ---- end to end through the public API, host buffers, copies inside the timing
+    h_out = {n: torch.empty(q.shape, dtype=tdt).pin_memory() for n in ("o", "dq", "dk", "dv")}
+    h_L = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values()) + h_L.numel() * 4
+
+    def e2e_step():
+        for n in ("q", "k", "v", "do"):
+            dv_in[n].copy_(h_in[n], non_blocking=True)
+        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, stream=stream)
+        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=scale, workspace=ws, dq=dq, dk=dk,
+                    dv=dvv, stream=stream)
+        for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv)):
+            h_out[n].copy_(t, non_blocking=True)
+        h_L.copy_(L, non_blocking=True)
+
+    if args.e2e_steps <= 0:
+        e2e_ms = float("nan")
+    else:
+        e2e_step()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    if args.e2e_steps > 0:
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_val = world * (2.5 * fwd_f) * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "fp16",
+        "data": "synthetic (seeded iid N(0,1), rounded to 16 bit)", "config": config_of(w),
+        "fwd_tflops": fwd_f / (fwd_ms * 1e-3) / 1e12,
+        "bwd_tflops": bwd_f / (bwd_ms * 1e-3) / 1e12,
+        "fwd_bwd_tflops_3p5x": world * (fwd_f + bwd_f) * steps / (total_ms * 1e-3) / 1e12,
+        "pct_of_peak": {"fwd": fwd_f / (fwd_ms * 1e-3) / 1e12 / peak_sus,
+                        "fwd_bwd_2p5x": value / world / peak_sus,
+                        "fwd_bwd_3p5x": (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12 / peak_sus,
+                        "peak": peak_sus, "peak_kind": f"{peak_kind} bf16 sustained"},
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                "api": "fa.forward + fa.backward (C ABI) with pinned host buffers"},
+        "gpu_launches": 4 * steps,
+        "clocks": clocks,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        outs = {"o": o.float().cpu().numpy(), "dq": dq.float().cpu().numpy(),
+                "dk": dk.float().cpu().numpy(), "dv": dvv.float().cpu().numpy(),
+                "L": L.cpu().numpy()}
+        base, parity = cpu_baseline_and_parity(w, inp, outs, args.cpu_seconds)
+        line["cpu_baseline"] = base
+        line["parity"] = parity
+        if not parity["ok"]:
+            log(json.dumps(line))
+            raise SystemExit("parity check of the timed outputs against the oracle FAILED")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

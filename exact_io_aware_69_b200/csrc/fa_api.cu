@@ -87,42 +87,61 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+struct BwdArgs {
+  const CUtensorMap* q;
+  const CUtensorMap* k;
+  const CUtensorMap* v;
+  const CUtensorMap* dO_map;
+  const void* O;
+  const void* dO;
+  const float* L;
+  void* dQ;
+  void* dK;
+  void* dV;
+  int BH;
+  int N;
+  float scale;
+  void* workspace;
+  cudaStream_t stream;
+};
+
+enum { kStagePre = 1, kStageMain = 2, kStageDq = 4, kStageAll = 7 };
+
+// Workspace: D [rows] fp32, Ls [rows] fp32, dQ accumulator [rows][d] fp32.
 template <int D, bool CAUSAL, bool BF16>
-int launch_bwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-               const CUtensorMap& dO_map, const void* O, const void* dO, const float* L,
-               void* dQ, void* dK, void* dV, int BH, int N, float scale, void* workspace,
-               cudaStream_t stream) {
-  const long rows = static_cast<long>(BH) * N;
-  float* Dv = static_cast<float*>(workspace);
+int launch_bwd(const BwdArgs& a, int stages) {
+  const long rows = static_cast<long>(a.BH) * a.N;
+  float* Dv = static_cast<float*>(a.workspace);
   float* Ls = Dv + rows;
   float* dq_acc = Ls + rows;
-  {
+  if (stages & kStagePre) {
     const long threads = rows * (D / 8);
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-    fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
-        static_cast<const uint16_t*>(O), static_cast<const uint16_t*>(dO), L, Dv, Ls, dq_acc,
-        rows);
+    fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
+        static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls,
+        dq_acc, rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  {
+  if (stages & kStageMain) {
     auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, BF16>;
     const size_t need = fa::BwdLayout<D>::kNeeded;
-    const size_t smem = need + 1024 <= kMaxDynSmem ? need + 1024 : kMaxDynSmem;
     if (need > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
+    const size_t smem = need + 1024 <= kMaxDynSmem ? need + 1024 : kMaxDynSmem;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return FA_ERR_CUDA;
-    const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
-    kern<<<grid, fa::kBwdThreads, smem, stream>>>(
-        q, k, v, dO_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(dK), static_cast<uint16_t*>(dV),
-        N, scale, scale * 1.4426950408889634074f, static_cast<uint32_t>(smem));
+    const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.N / fa::kTile);
+    kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
+        *a.q, *a.k, *a.v, *a.dO_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
+        static_cast<uint16_t*>(a.dV), a.N, a.scale, a.scale * 1.4426950408889634074f,
+        static_cast<uint32_t>(smem));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  {
+  if (stages & kStageDq) {
     const long n8 = rows * D / 8;
     const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
-    fa::fa_bwd_dq_kernel<D, BF16><<<blocks, 256, 0, stream>>>(dq_acc, static_cast<uint16_t*>(dQ),
-                                                             scale, n8);
+    fa::fa_bwd_dq_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
+        dq_acc, static_cast<uint16_t*>(a.dQ), a.scale, n8);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -194,26 +213,77 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4;
 }
 
+// Validation shared by fa_bwd and its stages; the pointers a stage does not use may
+// be NULL (checked by the caller).
+static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* workspace,
+               size_t workspace_bytes, bool* empty) {
+  int st = check_shape(B, H, N, d, dtype, scale, empty);
+  if (st != FA_OK || *empty) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID;
+  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID;
+  return FA_OK;
+}
+
+static int bwd_run(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+            const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+            int causal, float scale, int dtype, void* workspace, void* stream, int stages) {
+  const long rows = static_cast<long>(B) * H * N;
+  CUtensorMap tq, tk, tv, tdo;
+  if (stages & kStageMain) {
+    if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
+        !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype))
+      return FA_ERR_CUDA;
+  }
+  BwdArgs a{&tq, &tk, &tv, &tdo, O, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
+            static_cast<cudaStream_t>(stream)};
+  return dispatch<BwdRun>(d, causal, dtype, a, stages);
+}
+
+static bool ok_ptr(const void* p) { return p && aligned16(p); }
+
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
            const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal,
            float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   bool empty;
-  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
   if (st != FA_OK || empty) return st;
-  if (!Q || !K || !V || !O || !dO || !L || !dQ || !dK || !dV || !workspace)
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
+      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV))
     return FA_ERR_INVALID;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
-      !aligned16(L) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+  return bwd_run(Q, K, V, O, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype, workspace,
+                 stream, kStageAll);
+}
+
+int fa_bwd_preprocess(const void* O, const void* dO, const float* L, int B, int H, int N, int d,
+                      int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty;
+  int st = bwd_common(B, H, N, d, dtype, 1.f, workspace, workspace_bytes, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L)) return FA_ERR_INVALID;
+  return bwd_run(nullptr, nullptr, nullptr, O, dO, L, nullptr, nullptr, nullptr, B, H, N, d, 0,
+                 1.f, dtype, workspace, stream, kStagePre);
+}
+
+int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
+                int B, int H, int N, int d, int causal, float scale, int dtype, void* workspace,
+                size_t workspace_bytes, void* stream) {
+  bool empty;
+  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO) || !ok_ptr(dK) || !ok_ptr(dV))
     return FA_ERR_INVALID;
-  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID;
-  const long rows = static_cast<long>(B) * H * N;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
-      !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype))
-    return FA_ERR_CUDA;
-  return dispatch<BwdRun>(d, causal, dtype, tq, tk, tv, tdo, O, dO, L, dQ, dK, dV, B * H, N,
-                          scale, workspace, static_cast<cudaStream_t>(stream));
+  return bwd_run(Q, K, V, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, d, causal, scale,
+                 dtype, workspace, stream, kStageMain);
+}
+
+int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dtype,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty;
+  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!ok_ptr(dQ)) return FA_ERR_INVALID;
+  return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr, nullptr, B,
+                 H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
 }
 
 int fa_get_device_status(void* stream) {

@@ -30,6 +30,10 @@ SIGNATURES = {
     "fa_bwd_workspace_size": (_sz, [_int, _int, _int, _int]),
     "fa_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int,
                       _f32, _int, _vp, _sz, _vp]),
+    "fa_bwd_preprocess": (_int, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, _sz, _vp]),
+    "fa_bwd_dkdv": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32,
+                           _int, _vp, _sz, _vp]),
+    "fa_bwd_dq_convert": (_int, [_vp, _int, _int, _int, _int, _f32, _int, _vp, _sz, _vp]),
     "fa_get_device_status": (_int, [_vp]),
     "fa_status_string": (ctypes.c_char_p, [_int]),
     "fa_version": (_int, []),
@@ -140,6 +144,30 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
+
+
+def backward_stage(stage: str, q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool,
+                   scale: float, stream=None) -> None:
+    """Run one stage of the backward ("preprocess", "dkdv" or "dq_convert") on buffers
+    the caller already holds; the three in that order equal backward()."""
+    lib = load()
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    ws, wsb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    s = _stream_handle(stream)
+    if stage == "preprocess":
+        rc = lib.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, dt, ws,
+                                   wsb, s)
+    elif stage == "dkdv":
+        rc = lib.fa_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
+                             dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)),
+                             float(scale), dt, ws, wsb, s)
+    elif stage == "dq_convert":
+        rc = lib.fa_bwd_dq_convert(dq.data_ptr(), B, H, N, d, float(scale), dt, ws, wsb, s)
+    else:
+        raise ValueError(stage)
+    if rc != FA_OK:
+        raise FaError(rc, f"fa_bwd stage {stage}")
 
 
 def device_status(stream=None) -> int:

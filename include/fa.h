@@ -82,7 +82,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  * Backward. Given Q, K, V, the forward's O and L, and dO, writes dQ, dK, dV
  * ([B][H][N][d], dtype). `workspace` is a caller-owned device buffer of at least
  * fa_bwd_workspace_size(B, H, N, d) bytes, 256-byte aligned; its contents on entry
- * do not matter and on return are scratch. Four kernel launches: D = rowsum(dO * O)
+ * do not matter and on return are scratch. Three kernel launches: D = rowsum(dO * O)
  * and zeroing of the dQ accumulator; the dK/dV pass that recomputes P from L and
  * adds dQ partials atomically; the conversion of dQ to dtype.
  */
@@ -91,9 +91,29 @@ int fa_bwd(const void *Q, const void *K, const void *V, const void *O, const voi
            float scale, int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The three stages of fa_bwd, callable one by one (same arguments, same checks, same
+ * workspace; fa_bwd is exactly these three in this order on one stream). Each is one
+ * kernel launch.
+ *   fa_bwd_preprocess  D_i = sum_t dO_it O_it and L * log2(e) into the workspace,
+ *                      and zeroes its fp32 dQ accumulator.
+ *   fa_bwd_dkdv        recomputes P from Q, K and the workspace's scaled L, writes
+ *                      dK and dV, and adds the dQ partials into the accumulator.
+ *                      Needs fa_bwd_preprocess to have run on this workspace.
+ *   fa_bwd_dq_convert  dQ = dtype(scale * accumulator).
+ */
+int fa_bwd_preprocess(const void *O, const void *dO, const float *L, int B, int H, int N, int d,
+                      int dtype, void *workspace, size_t workspace_bytes, void *stream);
+int fa_bwd_dkdv(const void *Q, const void *K, const void *V, const void *dO, void *dK, void *dV,
+                int B, int H, int N, int d, int causal, float scale, int dtype, void *workspace,
+                size_t workspace_bytes, void *stream);
+int fa_bwd_dq_convert(void *dQ, int B, int H, int N, int d, float scale, int dtype,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of the
- * current device: FA_OK, or FA_ERR_TIMEOUT if a kernel abandoned a bounded wait.
- * FA_ERR_CUDA if the synchronisation itself failed.
+ * current device: FA_OK; FA_ERR_TIMEOUT if a kernel abandoned a bounded wait;
+ * FA_ERR_CUDA if the synchronisation failed or a kernel found its shared memory
+ * placed differently than it needs (it then returned without doing anything).
  */
 int fa_get_device_status(void *stream);
 
