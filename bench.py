@@ -287,6 +287,7 @@ def main():
     dv_in = {n: t.to(dev) for n, t in h_in.items()}
     q, k, v, do = dv_in["q"], dv_in["k"], dv_in["v"], dv_in["do"]
     o = torch.empty_like(q)
+    o_res = torch.empty_like(q)
     L = torch.empty((B, H, N), device=dev, dtype=torch.float32)
     dq, dk, dvv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws = torch.empty(fa.workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
@@ -295,16 +296,20 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, stream=stream)
+        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, out_res=o_res,
+                   stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        fa.backward_stage("preprocess", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        fa.backward_stage("preprocess", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale,
+                          o_res, stream)
         if ev is not None:
             ev[2].record(stream)
-        fa.backward_stage("dkdv", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        fa.backward_stage("dkdv", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, o_res,
+                          stream)
         if ev is not None:
             ev[3].record(stream)
-        fa.backward_stage("dq_convert", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale, stream)
+        fa.backward_stage("dq_convert", q, k, v, o, L, do, dq, dk, dvv, ws, w.causal, scale,
+                          o_res, stream)
         if ev is not None:
             ev[4].record(stream)
 
@@ -362,7 +367,7 @@ def main():
     # dominant kernel: the largest share of the step
     kflops = {"fa_fwd_kernel": fwd_f, "fa_bwd_main_kernel": bwd_f}
     rows = B * H * N
-    kbytes = {"fa_bwd_pre_kernel": rows * d * 2 * 2 + rows * 4 + rows * 8 + rows * d * 4,
+    kbytes = {"fa_bwd_pre_kernel": rows * d * 2 * 3 + rows * 4 + rows * 8 + rows * d * 4,
               "fa_bwd_dq_kernel": rows * d * 4 + rows * d * 2}
     dom = max(per_kernel, key=per_kernel.get)
     dom_ms = per_kernel[dom] / steps
@@ -401,8 +406,10 @@ def main():
     def e2e_step():
         for n in ("q", "k", "v", "do"):
             dv_in[n].copy_(h_in[n], non_blocking=True)
-        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, stream=stream)
-        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=scale, workspace=ws, dq=dq, dk=dk,
+        fa.forward(q, k, v, causal=w.causal, scale=scale, out=o, lse=L, out_res=o_res,
+                   stream=stream)
+        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=scale, o_res=o_res, workspace=ws,
+                    dq=dq, dk=dk,
                     dv=dvv, stream=stream)
         for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dvv)):
             h_out[n].copy_(t, non_blocking=True)

@@ -73,7 +73,7 @@ int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty)
 
 template <int D, bool CAUSAL, bool BF16>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, void* O,
-               float* L, int BH, int N, float scale, cudaStream_t stream) {
+               void* O_res, float* L, int BH, int N, float scale, cudaStream_t stream) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, BF16>;
   // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
   // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
@@ -82,7 +82,8 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
       cudaSuccess)
     return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, static_cast<uint16_t*>(O), L, N,
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, static_cast<uint16_t*>(O),
+                                                 static_cast<uint16_t*>(O_res), L, N,
                                                  scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -93,6 +94,7 @@ struct BwdArgs {
   const CUtensorMap* v;
   const CUtensorMap* dO_map;
   const void* O;
+  const void* O_res;
   const void* dO;
   const float* L;
   void* dQ;
@@ -118,8 +120,8 @@ int launch_bwd(const BwdArgs& a, int stages) {
     const long threads = rows * (D / 8);
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
-        static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls,
-        dq_acc, rows);
+        static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.O_res),
+        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stages & kStageMain) {
@@ -187,20 +189,21 @@ const char* fa_status_string(int status) {
   }
 }
 
-int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int N,
-           int d, int causal, float scale, int dtype, void* stream) {
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L, int B,
+           int H, int N, int d, int causal, float scale, int dtype, void* stream) {
   bool empty;
   int st = check_shape(B, H, N, d, dtype, scale, &empty);
   if (st != FA_OK || empty) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L) ||
+      !aligned16(O_res))
     return FA_ERR_INVALID;
   const long rows = static_cast<long>(B) * H * N;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
       !make_tmap(&tv, V, rows, d, dtype))
     return FA_ERR_CUDA;
-  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, O, L, B * H, N, scale,
+  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, O, O_res, L, B * H, N, scale,
                           static_cast<cudaStream_t>(stream));
 }
 
@@ -224,8 +227,8 @@ static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* 
   return FA_OK;
 }
 
-static int bwd_run(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-            const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+static int bwd_run(const void* Q, const void* K, const void* V, const void* O,
+            const void* O_res, const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
             int causal, float scale, int dtype, void* workspace, void* stream, int stages) {
   const long rows = static_cast<long>(B) * H * N;
   CUtensorMap tq, tk, tv, tdo;
@@ -234,34 +237,36 @@ static int bwd_run(const void* Q, const void* K, const void* V, const void* O, c
         !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype))
       return FA_ERR_CUDA;
   }
-  BwdArgs a{&tq, &tk, &tv, &tdo, O, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
+  BwdArgs a{&tq, &tk, &tv, &tdo, O, O_res, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
             static_cast<cudaStream_t>(stream)};
   return dispatch<BwdRun>(d, causal, dtype, a, stages);
 }
 
 static bool ok_ptr(const void* p) { return p && aligned16(p); }
 
-int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-           const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d, int causal,
-           float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
+           const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N,
+           int d, int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
+           void* stream) {
   bool empty;
   int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
-      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV))
+      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
     return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, O, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype, workspace,
-                 stream, kStageAll);
+  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype,
+                 workspace, stream, kStageAll);
 }
 
-int fa_bwd_preprocess(const void* O, const void* dO, const float* L, int B, int H, int N, int d,
-                      int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+int fa_bwd_preprocess(const void* O, const void* O_res, const void* dO, const float* L, int B,
+                      int H, int N, int d, int dtype, void* workspace, size_t workspace_bytes,
+                      void* stream) {
   bool empty;
   int st = bwd_common(B, H, N, d, dtype, 1.f, workspace, workspace_bytes, &empty);
   if (st != FA_OK || empty) return st;
-  if (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L)) return FA_ERR_INVALID;
-  return bwd_run(nullptr, nullptr, nullptr, O, dO, L, nullptr, nullptr, nullptr, B, H, N, d, 0,
-                 1.f, dtype, workspace, stream, kStagePre);
+  if (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) || !aligned16(O_res)) return FA_ERR_INVALID;
+  return bwd_run(nullptr, nullptr, nullptr, O, O_res, dO, L, nullptr, nullptr, nullptr, B, H, N,
+                 d, 0, 1.f, dtype, workspace, stream, kStagePre);
 }
 
 int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
@@ -272,8 +277,8 @@ int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, voi
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO) || !ok_ptr(dK) || !ok_ptr(dV))
     return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, d, causal, scale,
-                 dtype, workspace, stream, kStageMain);
+  return bwd_run(Q, K, V, nullptr, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, d, causal,
+                 scale, dtype, workspace, stream, kStageMain);
 }
 
 int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dtype,
@@ -282,8 +287,8 @@ int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dty
   int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(dQ)) return FA_ERR_INVALID;
-  return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr, nullptr, B,
-                 H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
+  return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
+                 nullptr, B, H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
 }
 
 int fa_get_device_status(void* stream) {

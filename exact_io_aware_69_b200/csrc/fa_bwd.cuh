@@ -9,32 +9,40 @@
 //   dQ = scale * dS K,   dK = scale * dS^T Q.
 //
 // Three kernels:
-//   fa_bwd_pre_kernel   D = rowsum(dO * O) (fp32), Ls = L * log2(e), dQacc = 0.
+//   fa_bwd_pre_kernel   D = rowsum(dO * (O + O_res)) (fp32; O_res is the forward's
+//                       rounding residual of O, optional), Ls = L * log2(e), dQacc = 0.
 //   fa_bwd_main_kernel  one CTA per 128-key tile j of one head: K_j, V_j stay in
 //                       shared memory, the CTA walks the query tiles i that see
 //                       them, accumulates dK_j and dV_j in TMEM, and adds each
 //                       dQ_i partial into the fp32 accumulator with vector atomics.
 //   fa_bwd_dq_kernel    dQ = dtype(scale * dQacc).
 //
-// Main-kernel warp roles (320 threads):
-//   warps 0-3  compute: thread r owns key row r (TMEM lane r). P^T row from S^T and
-//              L, dS^T row from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to
-//              shared memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
-//              dK_j / dV_j epilogue.
-//   warp 4     TMA producer: K_j, V_j once; Q_i, dO_i, Ls_i, D_i into a 2-stage ring.
-//   warp 5     MMA issuer (and TMEM owner), per query tile:
+// Main-kernel warp roles (448 threads; 14 warps keep 4 or fewer per SM sub-partition,
+// which leaves each thread up to 128 registers):
+//   warps 0-7  compute, in pairs: warps w and w+4 share TMEM lane quarter w % 4, so
+//              thread r of the pair owns key row r = 32 (w % 4) + lane; warp w < 4
+//              takes query columns 0-63, warp w+4 columns 64-127 (no row reduction
+//              is needed here: L and D are per query column). P^T from S^T and L,
+//              dS^T from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to shared
+//              memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
+//              dK_j / dV_j epilogue, each warp of the pair writing half the columns.
+//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, Ls_i, D_i into a 2-stage ring.
+//   warp 9     MMA issuer (and TMEM owner), per query tile:
 //                S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (SMEM x SMEM)
 //                dV += P^T dO_i                              (P^T from TMEM)
 //                dK += dS^T Q_i, dQ_i = dS K_j                (dS from SMEM)
-//   warps 6-9  dQ drain: thread owns query row (warp % 4) * 32 + lane; copies the
-//              dQ_i tile out of TMEM and adds it to the fp32 accumulator.
+//   warps 10-13 dQ drain: thread owns query row (warp % 4) * 32 + lane; copies the
+//              dQ_i tile out of TMEM 32 columns at a time and adds it to the fp32
+//              accumulator with 16-byte reduce-adds.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace fa {
 
-constexpr int kBwdThreads = 320;
+constexpr int kBwdThreads = 448;
+constexpr int kBwdProducerWarp = 8;
+constexpr int kBwdMmaWarp = 9;
 
 template <int D>
 struct BwdLayout {
@@ -78,8 +86,9 @@ enum : int {
 // One group of D/8 threads per row: 8 elements (16 bytes) per thread.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
-    fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
-                      const float* __restrict__ L, float* __restrict__ Dv,
+    fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ O_res,
+                      const uint16_t* __restrict__ dO, const float* __restrict__ L,
+                      float* __restrict__ Dv,
                       float* __restrict__ Ls, float* __restrict__ dq_acc, long rows) {
   constexpr int kTpr = D / 8;  // threads per row
   const long gid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -89,15 +98,19 @@ __global__ void __launch_bounds__(256)
   if (row < rows) {
     const uint4 o = *reinterpret_cast<const uint4*>(O + row * D + part * 8);
     const uint4 g = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
+    const uint4 res = O_res != nullptr ? *reinterpret_cast<const uint4*>(O_res + row * D + part * 8)
+                                       : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t* ow = reinterpret_cast<const uint32_t*>(&o);
+    const uint32_t* rw = reinterpret_cast<const uint32_t*>(&res);
     const uint32_t* gw = reinterpret_cast<const uint32_t*>(&g);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      float o0, o1, g0, g1;
+      float o0, o1, r0, r1, g0, g1;
       unpack2<BF16>(ow[e], o0, o1);
+      unpack2<BF16>(rw[e], r0, r1);
       unpack2<BF16>(gw[e], g0, g1);
-      acc = fmaf(o0, g0, acc);
-      acc = fmaf(o1, g1, acc);
+      acc = fmaf(o0 + r0, g0, acc);
+      acc = fmaf(o1 + r1, g1, acc);
     }
     float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
     z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -170,7 +183,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(kBbSFull), 1);
     mbar_init(bar(kBbDPFull), 1);
-    mbar_init(bar(kBbPFull), 128);
+    mbar_init(bar(kBbPFull), 256);
     mbar_init(bar(kBbDSFree), 1);
     mbar_init(bar(kBbDQFull), 1);
     mbar_init(bar(kBbDQEmpty), 128);
@@ -178,7 +191,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kBwdMmaWarp) {
     tmem_alloc(sbase + Lay::kTmemSlot, 512);
     tmem_relinquish();
   }
@@ -187,7 +200,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
 
-  if (warp == 4) {
+  if (warp == kBwdProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch(&tmQ);
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bulk_load(sbase + Lay::kDv + st * 512, Dv + qrow, 512, full);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_sq = idesc_f16_f32(kTile, kTile, BF16, false, false);  // S^T, dP^T
@@ -278,65 +291,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       mma_commit(bar(kBbDone));
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ----------------------------------------------------------------- compute
-    const int r = warp * 32 + lane;  // key row within the tile
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    uint8_t* sds_row = smem + Lay::kDS + r * 128;
+    const int quarter = warp & 3;
+    const int half = warp >> 2;
+    const int r = quarter * 32 + lane;  // key row within the tile
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint8_t* sds_row = smem + Lay::kDS + half * Lay::kChunkBytes + r * 128;
     const int sw = r & 7;
     bool ok = true;
-    for (int it = 0; it < niter; ++it) {
+    for (int it = 0; it < niter && ok; ++it) {
       const int st = it & 1;
       const uint32_t ph = static_cast<uint32_t>(it & 1);
       const bool diag = CAUSAL && (i_begin + it == j);
-      if (!mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) ||
-          !mbar_wait(bar(kBbSFull), ph, abort_flag)) { ok = false; break; }
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) &&
+                          mbar_wait(bar(kBbSFull), ph, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      const float* sL = reinterpret_cast<const float*>(smem + Lay::kL + st * 512);
-      const float* sD = reinterpret_cast<const float*>(smem + Lay::kDv + st * 512);
-      float p[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
-        uint32_t sr[32];
-        tmem_ld32(lane_base + Lay::tS + c * 32, sr);
+      const float* sL = reinterpret_cast<const float*>(smem + Lay::kL + st * 512) + half * 64;
+      const float* sD = reinterpret_cast<const float*>(smem + Lay::kDv + st * 512) + half * 64;
+      // Both halves load their S^T columns before either writes P^T: the packed P^T
+      // of the upper half (columns 32-63) lands on S^T columns of the lower half.
+      float p[64];
+      {
+        uint32_t sr[64];
+        tmem_ld32(lane_base + Lay::tS + half * 64, sr);
+        tmem_ld32(lane_base + Lay::tS + half * 64 + 32, sr + 32);
         tmem_wait_ld();
         reg_fence32(sr);
+        reg_fence32(sr + 32);
+#pragma unroll
+        for (int q = 0; q < 64; ++q) p[q] = __uint_as_float(sr[q]);
+      }
+      named_bar_sync(1 + quarter, 64);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int q = c * 32 + e;
-          float x = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, -sL[q]));
-          if (diag && q < r) x = 0.f;
+          const int q = c * 32 + e;  // query column within this half
+          float x = ex2_approx(fmaf(p[q], scale_log2, -sL[q]));
+          if (diag && half * 64 + q < r) x = 0.f;
           p[q] = x;
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(p[c * 32 + 2 * e], p[c * 32 + 2 * e + 1]);
-        tmem_st16(lane_base + Lay::tS + c * 16, pk);
+        tmem_st16(lane_base + Lay::tS + half * 32 + c * 16, pk);
       }
-      if (!mbar_wait(bar(kBbDPFull), ph, abort_flag)) { ok = false; break; }
-      if (it > 0 && !mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)) { ok = false; break; }
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kBbDPFull), ph, abort_flag) &&
+                                       (it == 0 || mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)));
+      if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t dr[32];
-        tmem_ld32(lane_base + Lay::tDP + c * 32, dr);
+        tmem_ld32(lane_base + Lay::tDP + half * 64 + c * 32, dr);
         tmem_wait_ld();
         reg_fence32(dr);
-        uint32_t ds[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int q = c * 32 + 2 * e;
-          const float a = p[q] * (__uint_as_float(dr[2 * e]) - sD[q]);
-          const float b = p[q + 1] * (__uint_as_float(dr[2 * e + 1]) - sD[q + 1]);
-          ds[e] = pack2<BF16>(a, b);
-        }
-        // queries c*32 .. c*32+31 = 16-byte units u0..u0+3 of swizzle column c/2
-        uint8_t* base = sds_row + (c >> 1) * Lay::kChunkBytes;
+        // queries half*64 + c*32 .. +31 = 16-byte units c*4 .. c*4+3 of swizzle column `half`
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int unit = ((c & 1) * 4 + u) ^ sw;
-          *reinterpret_cast<uint4*>(base + unit * 16) =
-              make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
+          uint32_t ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 8 * u + 2 * e;  // column within this 32-column chunk
+            const int q = c * 32 + k;
+            const float a = p[q] * (__uint_as_float(dr[k]) - sD[q]);
+            const float b = p[q + 1] * (__uint_as_float(dr[k + 1]) - sD[q + 1]);
+            ds[e] = pack2<BF16>(a, b);
+          }
+          const int unit = (c * 4 + u) ^ sw;
+          *reinterpret_cast<uint4*>(sds_row + unit * 16) = make_uint4(ds[0], ds[1], ds[2], ds[3]);
         }
       }
       fence_async_smem();
@@ -344,16 +370,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(bar(kBbPFull));
     }
-    if (ok && mbar_wait(bar(kBbDone), 0, abort_flag)) {
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBbDone), 0, abort_flag));
+    if (ok) {
       tc_fence_after();
       const long grow = head_row + static_cast<long>(j) * kTile + r;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? Lay::tDV : Lay::tDK;
+        const uint32_t col = (which == 0 ? Lay::tDV : Lay::tDK) + half * (D / 2);
         const float mul = which == 0 ? 1.f : scale;
-        uint16_t* dst_row = (which == 0 ? dV : dK) + grow * D;
+        uint16_t* dst_row = (which == 0 ? dV : dK) + grow * D + half * (D / 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
           tmem_ld32(lane_base + col + c * 32, v);
           tmem_wait_ld();
@@ -375,28 +402,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int qr = quarter * 32 + lane;  // query row within tile i
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     for (int it = 0; it < niter; ++it) {
-      if (!mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)) break;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)))
+        break;
       tc_fence_after();
-      uint32_t v[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar(kBbDQEmpty));
       float4* dst = reinterpret_cast<float4*>(
           dq_acc + (head_row + static_cast<long>(i_begin + it) * kTile + qr) * D);
 #pragma unroll
-      for (int e = 0; e < D / 4; ++e)
-        atomicAdd(dst + e, make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                       __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + Lay::tDQ + c * 32, v);
+        tmem_wait_ld();
+        reg_fence32(v);
+        if (c == D / 32 - 1) {
+          // the whole tile is out of TMEM: the MMA warp may overwrite it
+          tc_fence_before();
+          mbar_arrive(bar(kBbDQEmpty));
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          atomicAdd(dst + c * 8 + e,
+                    make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+      }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kBwdMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

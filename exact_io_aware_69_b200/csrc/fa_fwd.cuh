@@ -8,12 +8,15 @@
 // score and probability tiles live only in tensor memory (TMEM); Q, K, V are read
 // from HBM once per CTA ("una pasada sobre Q, K y V", same page, comparison table).
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r. Loads its score row
-//              from TMEM, masks, updates m and l, writes P (16-bit) back into TMEM
-//              over the scores, rescales its O row when m grew, and runs the epilogue.
-//   warp 4     TMA producer: Q once, then K_j / V_j into a 2-stage ring.
-//   warp 5     MMA issuer: S_j = Q K_j^T (SMEM x SMEM -> TMEM, fp32) and
+// Warp roles (320 threads):
+//   warps 0-7  softmax, in pairs: warps w and w+4 share TMEM lane quarter w % 4, so
+//              thread r of the pair's two warps owns query row r = 32 (w % 4) + lane;
+//              warp w < 4 takes score columns 0-63 and O columns [0, d/2), warp w+4
+//              columns 64-127 and [d/2, d). The pair exchanges its two partial row
+//              maxima through shared memory once per key tile; each half keeps its
+//              own partial row sum until the epilogue.
+//   warp 8     TMA producer: Q once, then K_j / V_j into a 2-stage ring.
+//   warp 9     MMA issuer: S_j = Q K_j^T (SMEM x SMEM -> TMEM, fp32) and
 //              O += P_j V_j (P from TMEM, V from SMEM -> TMEM, fp32). It also owns
 //              the TMEM allocation.
 //
@@ -24,14 +27,28 @@
 // Scores are kept in the base-2 domain: s' = s * scale * log2(e), p = 2^(s' - m').
 // The running reference m' is only moved when the row maximum exceeds it by more
 // than kRescaleSlack (so exponentials stay <= 2^kRescaleSlack); the result is the
-// same because l, O and L all share whatever reference is current.
+// same because l, O and L all share whatever reference is current. Two row sums
+// are kept: l_o adds up the 16-bit-rounded p, the very values the P V product
+// multiplies, and normalises O, so that O is an exact convex combination of V rows
+// with those weights (normalising by the unrounded sum would leave O off by up to
+// 2^-9 relative in every column at once for a row dominated by one key, and
+// D = rowsum(dO * O) in the backward would inherit that error); l adds up the
+// unrounded p and gives L, the log-sum-exp of the scores themselves.
+//
+// Optional second output O_res: the rounding residual of O in the same 16-bit type,
+// O_res = dtype(O_fp32 - O). O + O_res carries O to about 2^-17 relative, and the
+// backward uses it for D: a 16-bit O alone moves D_i by up to 2^-9 sum_t |dO_it O_it|,
+// and for a query row dominated by one key (large logits) dS_ij* = P (dP_ij* - D_i)
+// is a small difference that this error swamps.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace fa {
 
-constexpr int kFwdThreads = 192;
+constexpr int kFwdThreads = 320;
+constexpr int kFwdProducerWarp = 8;
+constexpr int kFwdMmaWarp = 9;
 constexpr float kRescaleSlack = 8.0f;
 
 template <int D>
@@ -41,7 +58,10 @@ struct FwdLayout {
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kTileBytes;        // 2 stages
   static constexpr uint32_t kV = kK + 2 * kTileBytes;    // 2 stages
-  static constexpr uint32_t kBar = kV + 2 * kTileBytes;
+  // [2 parity][2 half][128] fp32 row-max exchange; in the epilogue also [2][2][128]
+  // for the second row sum
+  static constexpr uint32_t kRed = kV + 2 * kTileBytes;
+  static constexpr uint32_t kBar = kRed + 2 * 2 * 2 * 128 * 4;
   static constexpr int kNumBars = 12;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 8;
@@ -63,7 +83,8 @@ template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, uint16_t* __restrict__ O,
-                  float* __restrict__ Lse, int N, float scale_log2) {
+                  uint16_t* __restrict__ O_res, float* __restrict__ Lse, int N,
+                  float scale_log2) {
   using Lay = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -90,13 +111,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarKVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), 128);
+      mbar_init(bar(kBarPFull + s), 256);
     }
     mbar_init(bar(kBarODone), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     tmem_alloc(sbase + Lay::kTmemSlot, 512);
     tmem_relinquish();
   }
@@ -105,7 +126,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
 
-  if (warp == 4) {
+  if (warp == kFwdProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch(&tmQ);
@@ -129,7 +150,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tma_load_2d(sv + c * Lay::kChunkBytes, &tmV, c * 64, krow, bar(kBarVFull + st));
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kFwdMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(kTile, kTile, BF16, false, false);
@@ -174,63 +195,80 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else {
     // ----------------------------------------------------------------- softmax
-    const int r = warp * 32 + lane;  // query row within the tile = TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m = -INFINITY;  // running reference, base-2 scaled units
-    float l = 0.f;
+    const int quarter = warp & 3;
+    const int half = warp >> 2;
+    const int r = quarter * 32 + lane;  // query row within the tile = TMEM lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t o_cols = 256 + half * (D / 2);
+    float* red = reinterpret_cast<float*>(smem + Lay::kRed);  // [parity][half][row]
+    const int pair_bar = 1 + quarter;                          // named barrier of the pair
+    float m = -INFINITY;  // running reference, base-2 scaled units (same in both halves)
+    float l = 0.f;        // this half's share of the row sum of p
+    float l_o = 0.f;      // ... and of the 16-bit-rounded p
+    // `ok` turns false (warp-uniformly) when a wait gives up; the loop then runs on
+    // without work so that both warps of a pair still meet at every named barrier.
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
       const int b = j & 1;
       const uint32_t use = static_cast<uint32_t>(j >> 1);
-      if (!mbar_wait(bar(kBarSFull + b), use & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[kTile];
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarSFull + b), use & 1, abort_flag));
+      float s[64];
+      float mx = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(lane_base + b * 128 + half * 64, sr);
+        tmem_ld32(lane_base + b * 128 + half * 64 + 32, sr + 32);
+        tmem_wait_ld();
+        reg_fence32(sr);
+        reg_fence32(sr + 32);
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) tmem_ld32(lane_base + b * 128 + c * 32, sr + c * 32);
-      tmem_wait_ld();
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
+        if (CAUSAL && j == t) {
 #pragma unroll
-      for (int c = 0; c < kTile / 32; ++c) reg_fence32(sr + c * 32);
-      float s[kTile];
+          for (int c = 0; c < 64; ++c)
+            if (half * 64 + c > r) s[c] = -INFINITY;
+        }
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) s[c] = __uint_as_float(sr[c]);
-      if (CAUSAL && j == t) {
-#pragma unroll
-        for (int c = 0; c < kTile; ++c)
-          if (c > r) s[c] = -INFINITY;
+        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < kTile; ++c) mx = fmaxf(mx, s[c]);
+      red[(b * 2 + half) * 128 + r] = mx;
+      named_bar_sync(pair_bar, 64);
+      mx = fmaxf(mx, red[(b * 2 + (half ^ 1)) * 128 + r]);
+      if (!ok) continue;
       const float cand = mx * scale_log2;
       const float m_new = (cand > m + kRescaleSlack) ? cand : m;
       const float alpha = ex2_approx(m - m_new);  // 0 on the first tile, 1 if unchanged
-      float rowsum = 0.f;
+      uint32_t pk[32];
+      float rowsum = 0.f, rowsum_o = 0.f;
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const float p = ex2_approx(fmaf(s[c], scale_log2, -m_new));
-        rowsum += p;
-        s[c] = p;
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2_approx(fmaf(s[2 * c], scale_log2, -m_new));
+        const float p1 = ex2_approx(fmaf(s[2 * c + 1], scale_log2, -m_new));
+        pk[c] = pack2<BF16>(p0, p1);
+        float r0, r1;
+        unpack2<BF16>(pk[c], r0, r1);
+        rowsum += p0 + p1;
+        rowsum_o += r0 + r1;
       }
       l = l * alpha + rowsum;
-      uint32_t pk[kTile / 2];
-#pragma unroll
-      for (int c = 0; c < kTile / 2; ++c) pk[c] = pack2<BF16>(s[2 * c], s[2 * c + 1]);
-      tmem_st32(lane_base + b * 128, pk);
-      tmem_st32(lane_base + b * 128 + 32, pk + 32);
+      l_o = l_o * alpha + rowsum_o;
+      tmem_st32(lane_base + b * 128 + half * 32, pk);
       if (j > 0) {
         // the previous P V must have landed before O is touched
-        if (!mbar_wait(bar(kBarODone), (j - 1) & 1, abort_flag)) { ok = false; break; }
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone), (j - 1) & 1, abort_flag));
+        if (!ok) continue;
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t o[32];
-            tmem_ld32(lane_base + 256 + c * 32, o);
+            tmem_ld32(lane_base + o_cols + c * 32, o);
             tmem_wait_ld();
             reg_fence32(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_base + 256 + c * 32, o);
+            tmem_st32(lane_base + o_cols + c * 32, o);
           }
         }
       }
@@ -239,32 +277,52 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_arrive(bar(kBarPFull + b));
       m = m_new;
     }
-    if (ok && mbar_wait(bar(kBarODone), (nkv - 1) & 1, abort_flag)) {
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarODone), (nkv - 1) & 1, abort_flag));
+    // both halves' sums: reuse the exchange buffer of parity (nkv & 1), which the pair
+    // last used two tiles ago
+    red[((nkv & 1) * 2 + half) * 128 + r] = l;
+    red[((nkv & 1) * 2 + half) * 128 + r + 512] = l_o;
+    named_bar_sync(pair_bar, 64);
+    const float l_row = l + red[((nkv & 1) * 2 + (half ^ 1)) * 128 + r];
+    const float l_o_row = l_o + red[((nkv & 1) * 2 + (half ^ 1)) * 128 + r + 512];
+    if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      uint16_t* orow = O + static_cast<size_t>(row0 + r) * D;
+      const float inv_l = 1.f / l_o_row;
+      const size_t obase = static_cast<size_t>(row0 + r) * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + 256 + c * 32, o);
+        tmem_ld32(lane_base + o_cols + c * 32, o);
         tmem_wait_ld();
         reg_fence32(o);
-        uint4 pkd[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pkd);
+        uint4 hi[4], lo[4];
+        uint32_t* hw = reinterpret_cast<uint32_t*>(hi);
+        uint32_t* lw = reinterpret_cast<uint32_t*>(lo);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pw[e] = pack2<BF16>(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = __uint_as_float(o[2 * e]) * inv_l;
+          const float x1 = __uint_as_float(o[2 * e + 1]) * inv_l;
+          hw[e] = pack2<BF16>(x0, x1);
+          float h0, h1;
+          unpack2<BF16>(hw[e], h0, h1);
+          lw[e] = pack2<BF16>(x0 - h0, x1 - h1);  // exact difference, then rounded
+        }
+        uint4* dst = reinterpret_cast<uint4*>(O + obase + c * 32);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = pkd[e];
+        for (int e = 0; e < 4; ++e) dst[e] = hi[e];
+        if (O_res != nullptr) {
+          uint4* dres = reinterpret_cast<uint4*>(O_res + obase + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dres[e] = lo[e];
+        }
       }
-      Lse[row0 + r] = (m + log2f(l)) * 0.69314718055994530942f;
+      if (half == 0) Lse[row0 + r] = (m + log2f(l_row)) * 0.69314718055994530942f;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kFwdMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -26,11 +26,13 @@ FA_FP16 = 1
 # Every symbol include/fa.h declares, with its ctypes signature.
 _vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
-    "fa_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32, _int, _vp]),
+    "fa_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32, _int,
+                      _vp]),
     "fa_bwd_workspace_size": (_sz, [_int, _int, _int, _int]),
-    "fa_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int,
-                      _f32, _int, _vp, _sz, _vp]),
-    "fa_bwd_preprocess": (_int, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, _sz, _vp]),
+    "fa_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
+                      _int, _f32, _int, _vp, _sz, _vp]),
+    "fa_bwd_preprocess": (_int, [_vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, _sz,
+                                 _vp]),
     "fa_bwd_dkdv": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32,
                            _int, _vp, _sz, _vp]),
     "fa_bwd_dq_convert": (_int, [_vp, _int, _int, _int, _int, _f32, _int, _vp, _sz, _vp]),
@@ -94,9 +96,16 @@ def _check(t, name, like=None):
         raise FaError(FA_ERR_INVALID, f"{name} shape/dtype differs from q")
 
 
+def _ptr_or_none(t):
+    return None if t is None else t.data_ptr()
+
+
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-            stream=None):
-    """O, L = attention(q, k, v) for [B, H, N, d] bf16/fp16 CUDA tensors."""
+            out_res=None, residual: bool = True, stream=None):
+    """(O, L, O_res) = attention(q, k, v) for [B, H, N, d] bf16/fp16 CUDA tensors.
+
+    O_res is the 16-bit rounding residual of O (None when residual=False); pass it to
+    backward() so that D = rowsum(dO * O) is formed from O at near-fp32 precision."""
     import torch
     lib = load()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -108,12 +117,14 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
-    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                    B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
-                    _stream_handle(stream))
+    if out_res is None and residual:
+        out_res = torch.empty_like(q)
+    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                    _ptr_or_none(out_res), lse.data_ptr(), B, H, N, d, int(bool(causal)),
+                    float(scale), _dtype_code(q), _stream_handle(stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
-    return out, lse
+    return out, lse, out_res
 
 
 def workspace_size(B, H, N, d) -> int:
@@ -121,8 +132,9 @@ def workspace_size(B, H, N, d) -> int:
 
 
 def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None,
-             workspace=None, dq=None, dk=None, dv=None, stream=None):
-    """dQ, dK, dV of attention, recomputing P from q, k, v and the forward's lse."""
+             o_res=None, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """dQ, dK, dV of attention, recomputing P from q, k, v and the forward's lse
+    (o_res: the forward's rounding residual of O, or None)."""
     import torch
     lib = load()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
@@ -137,8 +149,9 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
-    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr_or_none(o_res),
+                    do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                    B, H, N, d,
                     int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
                     workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != FA_OK:
@@ -147,7 +160,7 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
 
 
 def backward_stage(stage: str, q, k, v, o, lse, do, dq, dk, dv, workspace, causal: bool,
-                   scale: float, stream=None) -> None:
+                   scale: float, o_res=None, stream=None) -> None:
     """Run one stage of the backward ("preprocess", "dkdv" or "dq_convert") on buffers
     the caller already holds; the three in that order equal backward()."""
     lib = load()
@@ -156,8 +169,8 @@ def backward_stage(stage: str, q, k, v, o, lse, do, dq, dk, dv, workspace, causa
     ws, wsb = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     s = _stream_handle(stream)
     if stage == "preprocess":
-        rc = lib.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), lse.data_ptr(), B, H, N, d, dt, ws,
-                                   wsb, s)
+        rc = lib.fa_bwd_preprocess(o.data_ptr(), _ptr_or_none(o_res), do.data_ptr(),
+                                   lse.data_ptr(), B, H, N, d, dt, ws, wsb, s)
     elif stage == "dkdv":
         rc = lib.fa_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
                              dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(bool(causal)),

@@ -67,9 +67,15 @@ typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
 /*
  * Forward. Reads Q, K, V [B][H][N][d]; writes O [B][H][N][d] (dtype) and
  * L [B][H][N] (fp32). One kernel launch.
+ *
+ * O_res (optional, may be NULL; otherwise [B][H][N][d] dtype, 16-byte aligned)
+ * receives the rounding residual of O: O_res = dtype(O_exact_fp32 - O), so that
+ * O + O_res holds the output to about 2^-17 relative. fa_bwd uses it for
+ * D_i = sum_t dO_it O_it; without it D carries the 16-bit rounding of O, which for
+ * rows dominated by one key (large logits) moves dK by several 1e-2.
  */
-int fa_fwd(const void *Q, const void *K, const void *V, void *O, float *L, int B, int H, int N,
-           int d, int causal, float scale, int dtype, void *stream);
+int fa_fwd(const void *Q, const void *K, const void *V, void *O, void *O_res, float *L, int B,
+           int H, int N, int d, int causal, float scale, int dtype, void *stream);
 
 /*
  * Bytes of device workspace that fa_bwd needs for this shape: fp32 D and scaled L
@@ -79,30 +85,32 @@ int fa_fwd(const void *Q, const void *K, const void *V, void *O, float *L, int B
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
- * Backward. Given Q, K, V, the forward's O and L, and dO, writes dQ, dK, dV
- * ([B][H][N][d], dtype). `workspace` is a caller-owned device buffer of at least
+ * Backward. Given Q, K, V, the forward's O, O_res (NULL allowed: D then uses O
+ * alone) and L, and dO, writes dQ, dK, dV ([B][H][N][d], dtype). `workspace` is a caller-owned device buffer of at least
  * fa_bwd_workspace_size(B, H, N, d) bytes, 256-byte aligned; its contents on entry
  * do not matter and on return are scratch. Three kernel launches: D = rowsum(dO * O)
  * and zeroing of the dQ accumulator; the dK/dV pass that recomputes P from L and
  * adds dQ partials atomically; the conversion of dQ to dtype.
  */
-int fa_bwd(const void *Q, const void *K, const void *V, const void *O, const void *dO,
-           const float *L, void *dQ, void *dK, void *dV, int B, int H, int N, int d, int causal,
-           float scale, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+int fa_bwd(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
+           const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H, int N,
+           int d, int causal, float scale, int dtype, void *workspace, size_t workspace_bytes,
+           void *stream);
 
 /*
  * The three stages of fa_bwd, callable one by one (same arguments, same checks, same
  * workspace; fa_bwd is exactly these three in this order on one stream). Each is one
  * kernel launch.
- *   fa_bwd_preprocess  D_i = sum_t dO_it O_it and L * log2(e) into the workspace,
- *                      and zeroes its fp32 dQ accumulator.
+ *   fa_bwd_preprocess  D_i = sum_t dO_it (O_it + O_res_it) and L * log2(e) into the
+ *                      workspace, and zeroes its fp32 dQ accumulator.
  *   fa_bwd_dkdv        recomputes P from Q, K and the workspace's scaled L, writes
  *                      dK and dV, and adds the dQ partials into the accumulator.
  *                      Needs fa_bwd_preprocess to have run on this workspace.
  *   fa_bwd_dq_convert  dQ = dtype(scale * accumulator).
  */
-int fa_bwd_preprocess(const void *O, const void *dO, const float *L, int B, int H, int N, int d,
-                      int dtype, void *workspace, size_t workspace_bytes, void *stream);
+int fa_bwd_preprocess(const void *O, const void *O_res, const void *dO, const float *L, int B,
+                      int H, int N, int d, int dtype, void *workspace, size_t workspace_bytes,
+                      void *stream);
 int fa_bwd_dkdv(const void *Q, const void *K, const void *V, const void *dO, void *dK, void *dV,
                 int B, int H, int N, int d, int causal, float scale, int dtype, void *workspace,
                 size_t workspace_bytes, void *stream);

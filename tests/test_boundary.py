@@ -60,20 +60,23 @@ P = 0x7F0000000000
 
 
 def _fwd(lib, **kw):
-    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, L=P + 0x400000, B=1, H=1,
-             N=256, d=64, causal=0, scale=0.125, dtype=fa.FA_BF16, stream=None)
+    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, R=P + 0xa00000,
+             L=P + 0x400000, B=1, H=1, N=256, d=64, causal=0, scale=0.125, dtype=fa.FA_BF16,
+             stream=None)
     a.update(kw)
-    return lib.fa_fwd(a["Q"], a["K"], a["V"], a["O"], a["L"], a["B"], a["H"], a["N"], a["d"],
-                      a["causal"], a["scale"], a["dtype"], a["stream"])
+    return lib.fa_fwd(a["Q"], a["K"], a["V"], a["O"], a["R"], a["L"], a["B"], a["H"], a["N"],
+                      a["d"], a["causal"], a["scale"], a["dtype"], a["stream"])
 
 
 def _bwd(lib, **kw):
-    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, dO=P + 0x400000,
+    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, R=P + 0xa00000,
+             dO=P + 0x400000,
              L=P + 0x500000, dQ=P + 0x600000, dK=P + 0x700000, dV=P + 0x800000, B=1, H=1, N=256,
              d=64, causal=0, scale=0.125, dtype=fa.FA_BF16, ws=P + 0x900000, ws_bytes=1 << 30,
              stream=None)
     a.update(kw)
-    return lib.fa_bwd(a["Q"], a["K"], a["V"], a["O"], a["dO"], a["L"], a["dQ"], a["dK"], a["dV"],
+    return lib.fa_bwd(a["Q"], a["K"], a["V"], a["O"], a["R"], a["dO"], a["L"], a["dQ"], a["dK"],
+                      a["dV"],
                       a["B"], a["H"], a["N"], a["d"], a["causal"], a["scale"], a["dtype"], a["ws"],
                       a["ws_bytes"], a["stream"])
 
@@ -84,6 +87,7 @@ def _bwd(lib, **kw):
     (dict(B=-1), fa.FA_ERR_INVALID),
     (dict(N=-128), fa.FA_ERR_INVALID),
     (dict(K=P + 8), fa.FA_ERR_INVALID),
+    (dict(R=P + 0xa00004), fa.FA_ERR_INVALID),
     (dict(scale=0.0), fa.FA_ERR_INVALID),
     (dict(scale=float("nan")), fa.FA_ERR_INVALID),
     (dict(scale=float("inf")), fa.FA_ERR_INVALID),
@@ -104,6 +108,7 @@ def test_fwd_rejects_before_launch(lib, kw, code):
     (dict(ws=P + 0x900010), fa.FA_ERR_INVALID),  # workspace must be 256-byte aligned
     (dict(ws_bytes=1000), fa.FA_ERR_INVALID),
     (dict(dV=P + 0x800002), fa.FA_ERR_INVALID),
+    (dict(R=P + 0xa00008), fa.FA_ERR_INVALID),
     (dict(H=-2), fa.FA_ERR_INVALID),
     (dict(d=32), fa.FA_ERR_UNSUPPORTED),
     (dict(N=130), fa.FA_ERR_UNSUPPORTED),

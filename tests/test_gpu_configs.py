@@ -25,8 +25,8 @@ def _run(w):
     import torch
     inp = w.make()
     q, k, v, do = (to_device(getattr(inp, n), w.dtype) for n in ("q", "k", "v", "do"))
-    o, L = fa.forward(q, k, v, causal=w.causal, scale=w.scale)
-    dq, dk, dv = fa.backward(q, k, v, o, L, do, causal=w.causal, scale=w.scale)
+    o, L, o_res = fa.forward(q, k, v, causal=w.causal, scale=w.scale)
+    dq, dk, dv = fa.backward(q, k, v, o, L, do, causal=w.causal, scale=w.scale, o_res=o_res)
     torch.cuda.synchronize()
     assert fa.device_status() == fa.FA_OK
     BH = w.B * w.H

@@ -30,8 +30,8 @@ def _run(B, H, N, d, dtype, causal, seed, large_frac=0.0):
     inp = make_inputs(B, H, N, d, dtype, seed, large_frac=large_frac)
     scale = 1.0 / math.sqrt(d)
     q, k, v, do = (to_device(getattr(inp, n), dtype) for n in ("q", "k", "v", "do"))
-    o, L = fa.forward(q, k, v, causal=causal, scale=scale)
-    dq, dk, dv = fa.backward(q, k, v, o, L, do, causal=causal, scale=scale)
+    o, L, o_res = fa.forward(q, k, v, causal=causal, scale=scale)
+    dq, dk, dv = fa.backward(q, k, v, o, L, do, causal=causal, scale=scale, o_res=o_res)
     torch.cuda.synchronize()
     assert fa.device_status() == fa.FA_OK
     ref = oracle.attn_bwd(*(inp.widened(n) for n in ("q", "k", "v", "do")), causal, scale)
@@ -63,10 +63,10 @@ def test_repeat_runs_are_stable():
     import torch
     inp = make_inputs(1, 2, 512, 64, BF16, seed=9)
     q, k, v, do = (to_device(getattr(inp, n), BF16) for n in ("q", "k", "v", "do"))
-    o1, L1 = fa.forward(q, k, v, causal=True)
-    o2, L2 = fa.forward(q, k, v, causal=True)
-    g1 = fa.backward(q, k, v, o1, L1, do, causal=True)
-    g2 = fa.backward(q, k, v, o1, L1, do, causal=True)
+    o1, L1, r1 = fa.forward(q, k, v, causal=True)
+    o2, L2, r2 = fa.forward(q, k, v, causal=True)
+    g1 = fa.backward(q, k, v, o1, L1, do, causal=True, o_res=r1)
+    g2 = fa.backward(q, k, v, o1, L1, do, causal=True, o_res=r1)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(L1, L2)
     assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])  # dK, dV: no atomics
