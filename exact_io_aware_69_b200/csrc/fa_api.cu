@@ -51,6 +51,21 @@ bool make_tmap(CUtensorMap* map, const void* ptr, long rows, int d, int dtype) {
   return r == CUDA_SUCCESS;
 }
 
+// [rows, d] row-major fp32 tensor, box of 32 columns (128 bytes) x 128 rows,
+// 128-byte swizzle: the dQ accumulator, target of TMA reduce-adds.
+bool make_tmap_f32(CUtensorMap* map, const void* ptr, long rows, int d) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
+  cuuint32_t box[2] = {32, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Shape checks shared by fa_fwd and fa_bwd. Returns FA_OK to proceed, or an error;
@@ -93,6 +108,7 @@ struct BwdArgs {
   const CUtensorMap* k;
   const CUtensorMap* v;
   const CUtensorMap* dO_map;
+  const CUtensorMap* dq_map;
   const void* O;
   const void* O_res;
   const void* dO;
@@ -134,7 +150,7 @@ int launch_bwd(const BwdArgs& a, int stages) {
       return FA_ERR_CUDA;
     const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.N / fa::kTile);
     kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
-        *a.q, *a.k, *a.v, *a.dO_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
+        *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
         static_cast<uint16_t*>(a.dV), a.N, a.scale, a.scale * 1.4426950408889634074f,
         static_cast<uint32_t>(smem));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -231,13 +247,15 @@ static int bwd_run(const void* Q, const void* K, const void* V, const void* O,
             const void* O_res, const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
             int causal, float scale, int dtype, void* workspace, void* stream, int stages) {
   const long rows = static_cast<long>(B) * H * N;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (stages & kStageMain) {
+    const float* dq_acc = static_cast<const float*>(workspace) + 2 * rows;
     if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
-        !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype))
+        !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype) ||
+        !make_tmap_f32(&tdq, dq_acc, rows, d))
       return FA_ERR_CUDA;
   }
-  BwdArgs a{&tq, &tk, &tv, &tdo, O, O_res, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, O, O_res, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
             static_cast<cudaStream_t>(stream)};
   return dispatch<BwdRun>(d, causal, dtype, a, stages);
 }
@@ -290,6 +308,17 @@ int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dty
   return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
                  nullptr, B, H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
 }
+
+#ifdef FA_TRACE
+// Trace builds only: point the kernels at a device buffer of
+// kTraceSlots * kTraceIters * kTraceEvents uint64 and choose the CTAs to record.
+int fa_trace_attach(void* buf, const int* ctas) {
+  if (cudaMemcpyToSymbol(fa::g_fa_trace, &buf, sizeof(void*)) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(fa::g_fa_trace_cta, ctas, sizeof(int) * fa::kTraceSlots) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return FA_OK;
+}
+#endif
 
 int fa_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

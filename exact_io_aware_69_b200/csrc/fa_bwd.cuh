@@ -14,7 +14,7 @@
 //   fa_bwd_main_kernel  one CTA per 128-key tile j of one head: K_j, V_j stay in
 //                       shared memory, the CTA walks the query tiles i that see
 //                       them, accumulates dK_j and dV_j in TMEM, and adds each
-//                       dQ_i partial into the fp32 accumulator with vector atomics.
+//                       dQ_i partial into the fp32 accumulator with TMA reduce-adds.
 //   fa_bwd_dq_kernel    dQ = dtype(scale * dQacc).
 //
 // Main-kernel warp roles (448 threads; 14 warps keep 4 or fewer per SM sub-partition,
@@ -26,14 +26,16 @@
 //              dS^T from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to shared
 //              memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
 //              dK_j / dV_j epilogue, each warp of the pair writing half the columns.
-//   warp 8     TMA producer: K_j, V_j once; Q_i, dO_i, Ls_i, D_i into a 2-stage ring.
+//   warp 8     TMA producer: K_j, V_j once; Q_i, Ls_i, D_i into a 2-stage ring; dO_i
+//              into a single buffer (its last reader, the dV MMA, finishes well
+//              before the next dP^T MMA needs the next tile).
 //   warp 9     MMA issuer (and TMEM owner), per query tile:
 //                S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (SMEM x SMEM)
 //                dV += P^T dO_i                              (P^T from TMEM)
 //                dK += dS^T Q_i, dQ_i = dS K_j                (dS from SMEM)
 //   warps 10-13 dQ drain: thread owns query row (warp % 4) * 32 + lane; copies the
-//              dQ_i tile out of TMEM 32 columns at a time and adds it to the fp32
-//              accumulator with 16-byte reduce-adds.
+//              dQ_i tile out of TMEM, stages it in shared memory and has the TMA unit
+//              add it into the fp32 accumulator (cp.reduce.async.bulk.tensor).
 #pragma once
 
 #include "sm100.cuh"
@@ -51,10 +53,12 @@ struct BwdLayout {
   static constexpr uint32_t kK = 0;
   static constexpr uint32_t kV = kK + kTileBytes;
   static constexpr uint32_t kQ = kV + kTileBytes;       // 2 stages
-  static constexpr uint32_t kDO = kQ + 2 * kTileBytes;  // 2 stages
-  static constexpr uint32_t kDS = kDO + 2 * kTileBytes; // 128 keys x 128 queries, 16-bit
+  static constexpr uint32_t kDO = kQ + 2 * kTileBytes;  // 1 stage
+  static constexpr uint32_t kDS = kDO + kTileBytes;     // 128 keys x 128 queries, 16-bit
   static constexpr uint32_t kDSBytes = kTile * kTile * 2;
-  static constexpr uint32_t kL = kDS + kDSBytes;        // 2 stages x 128 fp32
+  static constexpr uint32_t kStage = kDS + kDSBytes;    // dQ staging: two 128 x 32 fp32 boxes
+  static constexpr uint32_t kStageBytes = 2 * kTile * 128;
+  static constexpr uint32_t kL = kStage + kStageBytes;  // 2 stages x 128 fp32
   static constexpr uint32_t kDv = kL + 2 * 512;         // 2 stages x 128 fp32
   static constexpr uint32_t kBar = kDv + 2 * 512;
   static constexpr int kNumBars = 16;
@@ -71,7 +75,7 @@ struct BwdLayout {
 
 enum : int {
   kBbKVFull = 0,
-  kBbQFull = 1,   // +stage
+  kBbQFull = 1,   // +stage (Q_i, Ls_i, D_i)
   kBbQEmpty = 3,  // +stage
   kBbSFull = 5,
   kBbDPFull = 6,
@@ -80,6 +84,8 @@ enum : int {
   kBbDQFull = 9,
   kBbDQEmpty = 10,
   kBbDone = 11,
+  kBbDOFull = 12,
+  kBbDOEmpty = 13,
 };
 
 // ------------------------------------------------------------------ preprocess
@@ -147,7 +153,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmDO, const float* __restrict__ Ls,
+                       const __grid_constant__ CUtensorMap tmDO,
+                       const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ Ls,
                        const float* __restrict__ Dv, float* __restrict__ dq_acc,
                        uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int N,
                        float scale, float scale_log2, uint32_t smem_alloc) {
@@ -188,6 +195,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(kBbDQFull), 1);
     mbar_init(bar(kBbDQEmpty), 128);
     mbar_init(bar(kBbDone), 1);
+    mbar_init(bar(kBbDOFull), 1);
+    mbar_init(bar(kBbDOEmpty), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -207,6 +216,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
       tma_prefetch(&tmDO);
+      tma_prefetch(&tmDQ);
       const int krow = static_cast<int>(head_row) + j * kTile;
       mbar_expect_tx(bar(kBbKVFull), 2 * Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
@@ -216,18 +226,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int it = 0; it < niter; ++it) {
         const int st = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
-        if (it >= 2 && !mbar_wait(bar(kBbQEmpty + st), (use - 1) & 1, abort_flag)) break;
         const int qrow = static_cast<int>(head_row) + (i_begin + it) * kTile;
+        if (it >= 2 && !mbar_wait(bar(kBbQEmpty + st), (use - 1) & 1, abort_flag)) break;
         const uint32_t full = bar(kBbQFull + st);
-        mbar_expect_tx(full, 2 * Lay::kTileBytes + 2 * 512);
-        for (int c = 0; c < D / 64; ++c) {
+        mbar_expect_tx(full, Lay::kTileBytes + 2 * 512);
+        for (int c = 0; c < D / 64; ++c)
           tma_load_2d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
                       qrow, full);
-          tma_load_2d(sbase + Lay::kDO + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmDO,
-                      c * 64, qrow, full);
-        }
         bulk_load(sbase + Lay::kL + st * 512, Ls + qrow, 512, full);
         bulk_load(sbase + Lay::kDv + st * 512, Dv + qrow, 512, full);
+        if (it >= 1 &&
+            !mbar_wait(bar(kBbDOEmpty), static_cast<uint32_t>((it - 1) & 1), abort_flag))
+          break;
+        mbar_expect_tx(bar(kBbDOFull), Lay::kTileBytes);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_2d(sbase + Lay::kDO + c * Lay::kChunkBytes, &tmDO, c * 64, qrow,
+                      bar(kBbDOFull));
+        FA_TRACE_EVENT(it, 0);
       }
     }
   } else if (warp == kBwdMmaWarp) {
@@ -243,8 +258,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         const uint32_t ph = static_cast<uint32_t>(it & 1);
         const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
-        const uint32_t sdo = sbase + Lay::kDO + st * Lay::kTileBytes;
+        const uint32_t sdo = sbase + Lay::kDO;
         if (!mbar_wait(bar(kBbQFull + st), use & 1, abort_flag)) break;
+        FA_TRACE_EVENT(it, 1);
         tc_fence_after();
         // S^T = K_j Q_i^T
 #pragma unroll
@@ -254,8 +270,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  id_sq, k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbSFull));
+        FA_TRACE_EVENT(it, 2);
         // dP^T = V_j dO_i^T, into columns the previous dQ tile may still occupy
         if (it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
+        if (!mbar_wait(bar(kBbDOFull), ph, abort_flag)) break;
+        FA_TRACE_EVENT(it, 3);
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
@@ -264,7 +283,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                  sdesc_sw128(sdo + off, 16, 1024), id_sq, k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbDPFull));
+        FA_TRACE_EVENT(it, 4);
         if (!mbar_wait(bar(kBbPFull), ph, abort_flag)) break;
+        FA_TRACE_EVENT(it, 5);
         tc_fence_after();
         // dV += P^T dO_i  (K = the 128 queries of tile i)
 #pragma unroll
@@ -272,6 +293,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8,
                  sdesc_sw128(sdo + k * 2048, Lay::kChunkBytes, 1024), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bar(kBbDOEmpty));  // dO_i has been read for the last time
         // dK += dS^T Q_i
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
@@ -288,6 +310,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(bar(kBbQEmpty + st));
         mma_commit(bar(kBbDSFree));
         mma_commit(bar(kBbDQFull));
+        FA_TRACE_EVENT(it, 6);
       }
       mma_commit(bar(kBbDone));
     }
@@ -308,6 +331,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) &&
                           mbar_wait(bar(kBbSFull), ph, abort_flag));
       if (!ok) break;
+      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 7);
       tc_fence_after();
       const float* sL = reinterpret_cast<const float*>(smem + Lay::kL + st * 512) + half * 64;
       const float* sD = reinterpret_cast<const float*>(smem + Lay::kDv + st * 512) + half * 64;
@@ -325,6 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int q = 0; q < 64; ++q) p[q] = __uint_as_float(sr[q]);
       }
       named_bar_sync(1 + quarter, 64);
+      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 8);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
@@ -339,9 +364,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(p[c * 32 + 2 * e], p[c * 32 + 2 * e + 1]);
         tmem_st16(lane_base + Lay::tS + half * 32 + c * 16, pk);
       }
+      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 9);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kBbDPFull), ph, abort_flag) &&
                                        (it == 0 || mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)));
       if (!ok) break;
+      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 10);
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -369,6 +396,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBbPFull));
+      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 11);
     }
     ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBbDone), 0, abort_flag));
     if (ok) {
@@ -398,34 +426,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else {
     // ---------------------------------------------------------------- dQ drain
+    // dQ_i leaves TMEM into registers (then the MMA warp may reuse the columns), is
+    // staged in shared memory in the 128-byte-swizzled layout of a 128-row x 32-column
+    // fp32 box, and is added into the fp32 accumulator by TMA reduce-adds that one
+    // thread issues. Before a round overwrites the staging buffer, that thread waits
+    // until the TMA unit has read the previous round.
     const int quarter = warp & 3;
     const int qr = quarter * 32 + lane;  // query row within tile i
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool leader = (warp == 10 && lane == 0);
+    const uint32_t stage = sbase + Lay::kStage;
+    uint8_t* stage_row = smem + Lay::kStage + qr * 128;
+    const int sw = qr & 7;
     for (int it = 0; it < niter; ++it) {
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)))
+      // the four drain warps decide together, so that all of them meet every named barrier
+      if (!named_bar_and(5, 128,
+                         mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)))
         break;
+      if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
       tc_fence_after();
-      float4* dst = reinterpret_cast<float4*>(
-          dq_acc + (head_row + static_cast<long>(i_begin + it) * kTile + qr) * D);
+      uint32_t v[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + Lay::tDQ + c * 32, v);
-        tmem_wait_ld();
-        reg_fence32(v);
-        if (c == D / 32 - 1) {
-          // the whole tile is out of TMEM: the MMA warp may overwrite it
-          tc_fence_before();
-          mbar_arrive(bar(kBbDQEmpty));
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
+      tc_fence_before();
+      mbar_arrive(bar(kBbDQEmpty));
+      if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
+      const int row = static_cast<int>(head_row) + (i_begin + it) * kTile;
+#pragma unroll
+      for (int rnd = 0; rnd < D / 64; ++rnd) {
+        if (leader) bulk_wait_read_all();  // previous round's boxes have been read
+        named_bar_sync(5, 128);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int box = 2 * rnd + h;  // columns 32 box .. 32 box + 31
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(stage_row + h * Lay::kChunkBytes + ((u ^ sw) * 16)) =
+                make_uint4(v[32 * box + 4 * u], v[32 * box + 4 * u + 1],
+                           v[32 * box + 4 * u + 2], v[32 * box + 4 * u + 3]);
         }
+        fence_async_smem();
+        named_bar_sync(5, 128);
+        if (leader) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          atomicAdd(dst + c * 8 + e,
-                    make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3])));
+          for (int h = 0; h < 2; ++h)
+            tma_reduce_add_2d(&tmDQ, stage + h * Lay::kChunkBytes, 32 * (2 * rnd + h), row);
+          bulk_commit();
+        }
       }
+      if (leader) FA_TRACE_EVENT(it, 14);
     }
+    if (leader) bulk_wait_all();  // every reduce-add has landed before the CTA exits
   }
 
   tc_fence_before();

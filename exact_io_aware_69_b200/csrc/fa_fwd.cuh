@@ -15,7 +15,10 @@
 //              columns 64-127 and [d/2, d). The pair exchanges its two partial row
 //              maxima through shared memory once per key tile; each half keeps its
 //              own partial row sum until the epilogue.
-//   warp 8     TMA producer: Q once, then K_j / V_j into a 2-stage ring.
+//   warp 8     TMA producer: Q once, then K_j into a 3-stage ring and V_j into a
+//              2-stage ring, K one tile ahead of V (S_j needs K_j a whole softmax
+//              earlier than P_j V_j needs V_j). A K stage is released as soon as its
+//              S MMA completes, a V stage when its P V MMA does.
 //   warp 9     MMA issuer: S_j = Q K_j^T (SMEM x SMEM -> TMEM, fp32) and
 //              O += P_j V_j (P from TMEM, V from SMEM -> TMEM, fp32). It also owns
 //              the TMEM allocation.
@@ -51,18 +54,21 @@ constexpr int kFwdProducerWarp = 8;
 constexpr int kFwdMmaWarp = 9;
 constexpr float kRescaleSlack = 8.0f;
 
+constexpr int kFwdKStages = 3;
+constexpr int kFwdVStages = 2;
+
 template <int D>
 struct FwdLayout {
   static constexpr uint32_t kTileBytes = kTile * D * 2;  // 128 rows x D 16-bit values
   static constexpr uint32_t kChunkBytes = kTile * 128;   // 128 rows x 64 values (one swizzle column)
   static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTileBytes;        // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTileBytes;    // 2 stages
+  static constexpr uint32_t kK = kQ + kTileBytes;
+  static constexpr uint32_t kV = kK + kFwdKStages * kTileBytes;
   // [2 parity][2 half][128] fp32 row-max exchange; in the epilogue also [2][2][128]
   // for the second row sum
-  static constexpr uint32_t kRed = kV + 2 * kTileBytes;
+  static constexpr uint32_t kRed = kV + kFwdVStages * kTileBytes;
   static constexpr uint32_t kBar = kRed + 2 * 2 * 2 * 128 * 4;
-  static constexpr int kNumBars = 12;
+  static constexpr int kNumBars = 16;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 8;
   static constexpr uint32_t kBytes = kAbort + 8 + 1024;  // + alignment slack
@@ -71,13 +77,16 @@ struct FwdLayout {
 // barrier indices
 enum : int {
   kBarQFull = 0,
-  kBarKFull = 1,   // +stage
-  kBarVFull = 3,   // +stage
-  kBarKVEmpty = 5, // +stage
-  kBarSFull = 7,   // +buffer
-  kBarPFull = 9,   // +buffer
-  kBarODone = 11,
+  kBarKFull = 1,                        // + K stage
+  kBarKEmpty = kBarKFull + kFwdKStages,  // + K stage
+  kBarVFull = kBarKEmpty + kFwdKStages,  // + V stage
+  kBarVEmpty = kBarVFull + kFwdVStages,  // + V stage
+  kBarSFull = kBarVEmpty + kFwdVStages,  // + S buffer
+  kBarPFull = kBarSFull + 2,             // + S buffer
+  kBarODone = kBarPFull + 2,
+  kFwdNumBars = kBarODone + 1,
 };
+static_assert(kFwdNumBars <= 16, "barrier area");
 
 template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -106,10 +115,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarQFull), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kFwdKStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < kFwdVStages; ++s) {
       mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarKVEmpty + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarPFull + s), 256);
     }
@@ -135,19 +149,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_expect_tx(bar(kBarQFull), Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c)
         tma_load_2d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, row0, bar(kBarQFull));
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        const uint32_t use = static_cast<uint32_t>(j >> 1);
-        if (j >= 2 && !mbar_wait(bar(kBarKVEmpty + st), (use - 1) & 1, abort_flag)) break;
-        const int krow = bh * N + j * kTile;
-        const uint32_t sk = sbase + Lay::kK + st * Lay::kTileBytes;
-        const uint32_t sv = sbase + Lay::kV + st * Lay::kTileBytes;
-        mbar_expect_tx(bar(kBarKFull + st), Lay::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sk + c * Lay::kChunkBytes, &tmK, c * 64, krow, bar(kBarKFull + st));
-        mbar_expect_tx(bar(kBarVFull + st), Lay::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sv + c * Lay::kChunkBytes, &tmV, c * 64, krow, bar(kBarVFull + st));
+      // step s loads K_s and V_{s-1}
+      for (int step = 0; step <= nkv; ++step) {
+        if (step < nkv) {
+          const int ks = step % kFwdKStages;
+          const uint32_t kuse = static_cast<uint32_t>(step / kFwdKStages);
+          if (step >= kFwdKStages &&
+              !mbar_wait(bar(kBarKEmpty + ks), (kuse - 1) & 1, abort_flag))
+            break;
+          const uint32_t sk = sbase + Lay::kK + ks * Lay::kTileBytes;
+          mbar_expect_tx(bar(kBarKFull + ks), Lay::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sk + c * Lay::kChunkBytes, &tmK, c * 64, bh * N + step * kTile,
+                        bar(kBarKFull + ks));
+          FA_TRACE_EVENT(step, 8);
+        }
+        if (step >= 1) {
+          const int j = step - 1;
+          const int vs = j % kFwdVStages;
+          const uint32_t vuse = static_cast<uint32_t>(j / kFwdVStages);
+          if (j >= kFwdVStages && !mbar_wait(bar(kBarVEmpty + vs), (vuse - 1) & 1, abort_flag))
+            break;
+          const uint32_t sv = sbase + Lay::kV + vs * Lay::kTileBytes;
+          mbar_expect_tx(bar(kBarVFull + vs), Lay::kTileBytes);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(sv + c * Lay::kChunkBytes, &tmV, c * 64, bh * N + j * kTile,
+                        bar(kBarVFull + vs));
+          FA_TRACE_EVENT(j, 9);
+        }
       }
     }
   } else if (warp == kFwdMmaWarp) {
@@ -159,28 +188,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = mbar_wait(bar(kBarQFull), 0, abort_flag);
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {
-          const int st = j & 1;
-          const uint32_t use = static_cast<uint32_t>(j >> 1);
-          if (!mbar_wait(bar(kBarKFull + st), use & 1, abort_flag)) break;
+          const int ks = j % kFwdKStages;
+          const uint32_t kuse = static_cast<uint32_t>(j / kFwdKStages);
+          if (!mbar_wait(bar(kBarKFull + ks), kuse & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t sk = sbase + Lay::kK + st * Lay::kTileBytes;
-          const uint32_t d_s = tmem + st * 128;
+          const uint32_t sk = sbase + Lay::kK + ks * Lay::kTileBytes;
+          const uint32_t d_s = tmem + (j & 1) * 128;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
             mma_ss(d_s, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc_s,
                    k > 0 ? 1u : 0u);
           }
-          mma_commit(bar(kBarSFull + st));
+          mma_commit(bar(kBarKEmpty + ks));
+          mma_commit(bar(kBarSFull + (j & 1)));
+          FA_TRACE_EVENT(j, 0);
         }
         if (j >= 1) {
           const int jj = j - 1;
           const int b = jj & 1;
-          const uint32_t use = static_cast<uint32_t>(jj >> 1);
-          if (!mbar_wait(bar(kBarPFull + b), use & 1, abort_flag)) break;
-          if (!mbar_wait(bar(kBarVFull + b), use & 1, abort_flag)) break;
+          const int vs = jj % kFwdVStages;
+          if (!mbar_wait(bar(kBarPFull + b), static_cast<uint32_t>(jj >> 1) & 1, abort_flag)) break;
+          FA_TRACE_EVENT(jj, 1);
+          if (!mbar_wait(bar(kBarVFull + vs), static_cast<uint32_t>(jj / kFwdVStages) & 1,
+                         abort_flag))
+            break;
           tc_fence_after();
-          const uint32_t sv = sbase + Lay::kV + b * Lay::kTileBytes;
+          const uint32_t sv = sbase + Lay::kV + vs * Lay::kTileBytes;
           const uint32_t a_p = tmem + b * 128;  // P packed in the first 64 columns
           const uint32_t d_o = tmem + 256;
 #pragma unroll
@@ -188,8 +222,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mma_ts(d_o, a_p + k * 8, sdesc_sw128(sv + k * 2048, Lay::kChunkBytes, 1024), idesc_o,
                    (jj > 0 || k > 0) ? 1u : 0u);
           }
-          mma_commit(bar(kBarKVEmpty + b));
+          mma_commit(bar(kBarVEmpty + vs));
           mma_commit(bar(kBarODone));
+          FA_TRACE_EVENT(jj, 2);
         }
       }
     }
@@ -212,6 +247,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int b = j & 1;
       const uint32_t use = static_cast<uint32_t>(j >> 1);
       ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarSFull + b), use & 1, abort_flag));
+      if (threadIdx.x == 0) FA_TRACE_EVENT(j, 3);
       float s[64];
       float mx = -INFINITY;
       if (ok) {
@@ -224,40 +260,55 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         reg_fence32(sr + 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        if (CAUSAL && j == t) {
+        if (CAUSAL && j == t) {  // diagonal tile: key column > query row is masked
+          const int lim = r - half * 64;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (half * 64 + c > r) s[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
         }
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
       }
       red[(b * 2 + half) * 128 + r] = mx;
       named_bar_sync(pair_bar, 64);
       mx = fmaxf(mx, red[(b * 2 + (half ^ 1)) * 128 + r]);
+      if (threadIdx.x == 0) FA_TRACE_EVENT(j, 4);
       if (!ok) continue;
       const float cand = mx * scale_log2;
       const float m_new = (cand > m + kRescaleSlack) ? cand : m;
       const float alpha = ex2_approx(m - m_new);  // 0 on the first tile, 1 if unchanged
-      uint32_t pk[32];
-      float rowsum = 0.f, rowsum_o = 0.f;
+      // pairs of lanes in packed fp32 (x2) arithmetic: argument, sums
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
+      const uint64_t nm2 = f2_pack(-m_new, -m_new);
+      uint64_t sum2 = 0, sum2_o = 0;  // two packed +0.0f
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], scale_log2, -m_new));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], scale_log2, -m_new));
-        pk[c] = pack2<BF16>(p0, p1);
-        float r0, r1;
-        unpack2<BF16>(pk[c], r0, r1);
-        rowsum += p0 + p1;
-        rowsum_o += r0 + r1;
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int e = h2 * 32 + 2 * c;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nm2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          pk[c] = pack2<BF16>(p0, p1);
+          float r0, r1;
+          unpack2<BF16>(pk[c], r0, r1);
+          sum2 = f2_add(sum2, f2_pack(p0, p1));
+          sum2_o = f2_add(sum2_o, f2_pack(r0, r1));
+        }
+        tmem_st16(lane_base + b * 128 + half * 32 + h2 * 16, pk);
       }
-      l = l * alpha + rowsum;
-      l_o = l_o * alpha + rowsum_o;
-      tmem_st32(lane_base + b * 128 + half * 32, pk);
+      float a0, a1, b0, b1;
+      f2_unpack(sum2, a0, a1);
+      f2_unpack(sum2_o, b0, b1);
+      l = l * alpha + (a0 + a1);
+      l_o = l_o * alpha + (b0 + b1);
+      if (threadIdx.x == 0) FA_TRACE_EVENT(j, 5);
       if (j > 0) {
         // the previous P V must have landed before O is touched
         ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone), (j - 1) & 1, abort_flag));
         if (!ok) continue;
+        if (threadIdx.x == 0) FA_TRACE_EVENT(j, 6);
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -275,6 +326,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarPFull + b));
+      if (threadIdx.x == 0) FA_TRACE_EVENT(j, 7);
       m = m_new;
     }
     ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarODone), (nkv - 1) & 1, abort_flag));

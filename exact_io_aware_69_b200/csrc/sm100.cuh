@@ -25,6 +25,28 @@ constexpr int kTile = 128;
 // Roughly 2 s at 2 GHz: a wait that has not completed by then will never complete.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+// ------------------------------------------------------------------ tracing
+// Built only with -DFA_TRACE (never in the product library): selected CTAs record
+// SM-clock timestamps of pipeline events into a caller-supplied device buffer laid
+// out [slot][iteration][event], so that a host script can draw each role's timeline.
+constexpr int kTraceSlots = 4;
+constexpr int kTraceIters = 128;
+constexpr int kTraceEvents = 16;
+#ifdef FA_TRACE
+__device__ unsigned long long* g_fa_trace = nullptr;
+__device__ int g_fa_trace_cta[kTraceSlots] = {-1, -1, -1, -1};
+__device__ __forceinline__ void trace_event(int it, int ev) {
+  if (g_fa_trace == nullptr || it < 0 || it >= kTraceIters) return;
+#pragma unroll
+  for (int s = 0; s < kTraceSlots; ++s)
+    if (g_fa_trace_cta[s] == static_cast<int>(blockIdx.x))
+      g_fa_trace[(s * kTraceIters + it) * kTraceEvents + ev] = clock64();
+}
+#define FA_TRACE_EVENT(it, ev) ::fa::trace_event((it), (ev))
+#else
+#define FA_TRACE_EVENT(it, ev) ((void)0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -93,6 +115,27 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
           "r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+// 2-D tiled reduce-add shared -> global (fp32 add done by the TMA unit / L2), in the
+// calling thread's bulk group.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32_t src, int x,
+                                                  int y) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk group of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor cores, TMA).
@@ -233,12 +276,79 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Named barrier that also ANDs a predicate over its `count` threads: every thread gets
+// true only if all passed true (a group-wide vote, e.g. on whether a wait succeeded).
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %3, 0;\n\t"
+      "bar.red.and.pred q, %1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------ arithmetic
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA/ALU pipes, without the MUFU unit (whose instructions share the
+// MIO issue queue with tcgen05.mma: a warp flooding it with ex2 starves the MMA
+// issuer on the same SM sub-partition). Cody-Waite style range reduction (Cody and
+// Waite, "Software Manual for the Elementary Functions", 1980): x = j + f with
+// j = round(x), obtained by adding 1.5 * 2^23 so that the low mantissa bits of the sum
+// hold j, and f = x - j in [-1/2, 1/2] exactly. 2^f comes from a degree-3 polynomial
+// whose coefficients were fitted for this kernel (weighted least squares on Chebyshev
+// nodes, minimising relative error: max 7.5e-5 on [-1/2, 1/2] in fp32 Horner form,
+// well below the 2^-9 / 2^-12 rounding of the 16-bit P it feeds); 2^j is added into
+// the exponent field: (bits of the shifted sum) << 23 equals j << 23 modulo 2^32.
+// Inputs below -125 are clamped (2^-125 is nothing next to a row sum >= 2^-8).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.05517161f, f, 0.24261111f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Packed fp32 pairs (sm_100): one instruction for two lanes of arithmetic.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// max of three
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Two floats -> packed 16-bit pair, round-to-nearest-even; `lo` lands in bits 0-15.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
