@@ -188,6 +188,38 @@ struct BwdRun {
   static int run(A&&... a) { return launch_bwd<D, C, B>(a...); }
 };
 
+// ------------------------------------------------ backward without allocation
+// Scratch of fa_bwd_noalloc: a fixed device array that every GPU loading this
+// library holds until the process exits. 32 MiB covers the backward workspace of
+// B*H*N up to 64,527 rows at d = 128 (128,100 rows at d = 64).
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device. Host code only sees a
+// host-side stand-in under that name, so the address is looked up once per device
+// (with that device current) and cached.
+constexpr int kMaxDevices = 64;
+void* noalloc_scratch_address(int* status) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *status = FA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      *status = FA_ERR_CUDA;
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *status = FA_OK;
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -307,6 +339,27 @@ int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dty
   if (!ok_ptr(dQ)) return FA_ERR_INVALID;
   return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
                  nullptr, B, H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
+}
+
+int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                   const void* O_res, const void* dO, const float* L, void* dQ, void* dK,
+                   void* dV, int B, int H, int N, int d, int causal, float scale, int dtype,
+                   void* stream) {
+  // Same checks as fa_bwd, and the size limit first: nothing touches the device for
+  // a problem that does not fit.
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need == static_cast<size_t>(-1)) return FA_ERR_INVALID;
+  if (need > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  bool empty;
+  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
+      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
+    return FA_ERR_INVALID;
+  void* scratch = noalloc_scratch_address(&st);
+  if (st != FA_OK) return st;
+  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype,
+                 scratch, stream, kStageAll);
 }
 
 #ifdef FA_TRACE

@@ -118,6 +118,33 @@ int fa_bwd_dq_convert(void *dQ, int B, int H, int N, int d, float scale, int dty
                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Backward without any device allocation. (The pages have no counterpart to this
+ * call: it is an interface convenience.) Some callers cannot allocate device memory
+ * at the point where they run the backward -- for instance a plugin inside a host
+ * application whose allocator owns the whole device, or a service that must not
+ * block or fail on an allocation in its steady state -- and so cannot provide the
+ * workspace fa_bwd wants. This variant takes the same arguments as fa_bwd minus the
+ * workspace and uses a fixed scratch array that is part of the library instead:
+ * 32 MiB, held on every GPU that loads the library until the process exits. It
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * Limit: fa_bwd_workspace_size(B, H, N, d) <= 32 MiB, i.e. B*H*N <= 64,527 at
+ * d = 128 and <= 128,100 at d = 64; larger problems return FA_ERR_UNSUPPORTED
+ * before anything touches the device. Other checks and results are those of
+ * fa_bwd.
+ *
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that first
+ * call before any stream capture. All calls on a device share the one array: the
+ * part that must start at zero (the dQ accumulator) is cleared by every call, but
+ * two calls whose work overlaps on the GPU (different streams, no ordering between
+ * them) race on it and give wrong gradients. Order such calls on one stream.
+ */
+int fa_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
+                   const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H,
+                   int N, int d, int causal, float scale, int dtype, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device error word of the
  * current device: FA_OK; FA_ERR_TIMEOUT if a kernel abandoned a bounded wait;
  * FA_ERR_CUDA if the synchronisation failed or a kernel found its shared memory

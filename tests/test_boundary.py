@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     assert names == sorted(["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_status",
                             "fa_status_string", "fa_version", "fa_bwd_preprocess",
-                            "fa_bwd_dkdv", "fa_bwd_dq_convert"])
+                            "fa_bwd_dkdv", "fa_bwd_dq_convert", "fa_bwd_noalloc"])
 
 
 def test_every_declared_symbol_is_exported(lib):
