@@ -79,13 +79,14 @@ enum : int {
   kBbQEmpty = 3,  // +stage
   kBbSFull = 5,
   kBbDPFull = 6,
-  kBbPFull = 7,
+  kBbPReady = 7,
   kBbDSFree = 8,
   kBbDQFull = 9,
   kBbDQEmpty = 10,
   kBbDone = 11,
   kBbDOFull = 12,
   kBbDOEmpty = 13,
+  kBbDSReady = 14,
 };
 
 // ------------------------------------------------------------------ preprocess
@@ -190,7 +191,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(kBbSFull), 1);
     mbar_init(bar(kBbDPFull), 1);
-    mbar_init(bar(kBbPFull), 256);
+    mbar_init(bar(kBbPReady), 256);
+    mbar_init(bar(kBbDSReady), 256);
     mbar_init(bar(kBbDSFree), 1);
     mbar_init(bar(kBbDQFull), 1);
     mbar_init(bar(kBbDQEmpty), 128);
@@ -247,22 +249,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
+    // Software-pipelined over the query tiles: with G1 = S^T, G2 = dP^T, G3 = dV,
+    // G4 = dK, G5 = dQ, the issue order is
+    //   G1(0) G2(0) | G3(0) G1(1) G4(0) G5(0) G2(1) | G3(1) G1(2) G4(1) G5(1) G2(2) | ...
+    // so that S^T of the next tile is computed while the compute warps form dS of the
+    // current one, and dK/dQ of the current tile while they exponentiate the next.
+    // G1(i+1) overwrites the S^T/P^T columns only after G3(i), which reads P^T, has
+    // been issued (MMAs from one thread execute in issue order).
     if (lane == 0) {
       constexpr uint32_t id_sq = idesc_f16_f32(kTile, kTile, BF16, false, false);  // S^T, dP^T
       constexpr uint32_t id_acc = idesc_f16_f32(kTile, D, BF16, false, true);      // dV, dK
       constexpr uint32_t id_dq = idesc_f16_f32(kTile, D, BF16, true, true);        // dQ
       const uint32_t sk = sbase + Lay::kK, sv = sbase + Lay::kV, sds = sbase + Lay::kDS;
-      bool ok = mbar_wait(bar(kBbKVFull), 0, abort_flag);
-      for (int it = 0; ok && it < niter; ++it) {
+      const uint32_t sdo = sbase + Lay::kDO;
+      auto issue_s = [&](int it) -> bool {  // G1: S^T = K_j Q_i^T
         const int st = it & 1;
-        const uint32_t use = static_cast<uint32_t>(it >> 1);
-        const uint32_t ph = static_cast<uint32_t>(it & 1);
-        const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
-        const uint32_t sdo = sbase + Lay::kDO;
-        if (!mbar_wait(bar(kBbQFull + st), use & 1, abort_flag)) break;
-        FA_TRACE_EVENT(it, 1);
+        if (!mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag))
+          return false;
         tc_fence_after();
-        // S^T = K_j Q_i^T
+        const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
@@ -271,10 +276,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit(bar(kBbSFull));
         FA_TRACE_EVENT(it, 2);
-        // dP^T = V_j dO_i^T, into columns the previous dQ tile may still occupy
-        if (it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
-        if (!mbar_wait(bar(kBbDOFull), ph, abort_flag)) break;
-        FA_TRACE_EVENT(it, 3);
+        return true;
+      };
+      auto issue_dp = [&](int it) -> bool {  // G2: dP^T = V_j dO_i^T
+        if (!mbar_wait(bar(kBbDOFull), static_cast<uint32_t>(it & 1), abort_flag)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
@@ -284,16 +289,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit(bar(kBbDPFull));
         FA_TRACE_EVENT(it, 4);
-        if (!mbar_wait(bar(kBbPFull), ph, abort_flag)) break;
+        return true;
+      };
+      bool ok = mbar_wait(bar(kBbKVFull), 0, abort_flag) && issue_s(0) && issue_dp(0);
+      for (int it = 0; ok && it < niter; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it & 1);
+        const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
+        // G3: dV += P^T dO_i (K = the 128 queries of tile i), P^T from TMEM
+        if (!mbar_wait(bar(kBbPReady), ph, abort_flag)) break;
         FA_TRACE_EVENT(it, 5);
         tc_fence_after();
-        // dV += P^T dO_i  (K = the 128 queries of tile i)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
           mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8,
                  sdesc_sw128(sdo + k * 2048, Lay::kChunkBytes, 1024), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar(kBbDOEmpty));  // dO_i has been read for the last time
+        FA_TRACE_EVENT(it, 3);
+        if (it + 1 < niter && !issue_s(it + 1)) break;
+        // G4, G5 once dS_i is in shared memory
+        if (!mbar_wait(bar(kBbDSReady), ph, abort_flag)) break;
+        FA_TRACE_EVENT(it, 1);
+        if (D != 128 && it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
+        tc_fence_after();
         // dK += dS^T Q_i
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
@@ -311,6 +330,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(bar(kBbDSFree));
         mma_commit(bar(kBbDQFull));
         FA_TRACE_EVENT(it, 6);
+        if (it + 1 < niter) {
+          // G2 of the next tile. At d = 128 its columns hold dQ_i until the drain has
+          // copied it out.
+          if (D == 128 && !mbar_wait(bar(kBbDQEmpty), ph, abort_flag)) break;
+          if (!issue_dp(it + 1)) break;
+        }
       }
       mma_commit(bar(kBbDone));
     }
@@ -364,6 +389,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(p[c * 32 + 2 * e], p[c * 32 + 2 * e + 1]);
         tmem_st16(lane_base + Lay::tS + half * 32 + c * 16, pk);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBbPReady));  // P^T is in TMEM: the dV MMA may go
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 9);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kBbDPFull), ph, abort_flag) &&
                                        (it == 0 || mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)));
@@ -393,9 +421,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       fence_async_smem();
-      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBbPFull));
+      mbar_arrive(bar(kBbDSReady));  // dS^T is in shared memory: dK and dQ may go
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 11);
     }
     ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBbDone), 0, abort_flag));
