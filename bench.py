@@ -175,6 +175,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(world, flops_per_rank_step, steps, max_ms):
+    """Whole-job rate: the work of all ranks over the slowest rank's time (TFLOP/s)."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def run_reference(args, w, rank):
     """The oracle as it stands, timed on this host's cores (rank 0 only)."""
     if rank != 0:
@@ -343,12 +358,10 @@ def main():
     for ev in events:
         for i, n in enumerate(names):
             per_kernel[n] += ev[i].elapsed_time(ev[i + 1])
-    if pg:
-        t = torch.tensor([total_ms] + [per_kernel[n] for n in names], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t[0])
-        for i, n in enumerate(names):
-            per_kernel[n] = float(t[1 + i])
+    red = max_over_ranks([total_ms] + [per_kernel[n] for n in names], pg, dev)
+    total_ms = red[0]
+    for i, n in enumerate(names):
+        per_kernel[n] = red[1 + i]
     st = fa.device_status()
     if st != fa.FA_OK:
         raise RuntimeError(f"device status {st} after timing")
@@ -357,7 +370,7 @@ def main():
     steps = args.steps
     ms_step = total_ms / steps
     # fwd+bwd counted as 2.5 x fwd, literally as the target states it
-    value = world * (2.5 * fwd_f) * steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(world, 2.5 * fwd_f, steps, total_ms)
     fwd_ms = per_kernel["fa_fwd_kernel"] / steps
     bwd_ms = sum(per_kernel[n] for n in names[1:]) / steps
     peaks, peak_kind = load_peaks()
@@ -431,11 +444,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_val = world * (2.5 * fwd_f) * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks([e2e_ms], pg, dev)[0]
+    e2e_val = job_throughput(world, 2.5 * fwd_f, args.e2e_steps, e2e_ms)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -444,7 +454,7 @@ def main():
         "data": "synthetic (seeded iid N(0,1), rounded to 16 bit)", "config": config_of(w),
         "fwd_tflops": fwd_f / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": bwd_f / (bwd_ms * 1e-3) / 1e12,
-        "fwd_bwd_tflops_3p5x": world * (fwd_f + bwd_f) * steps / (total_ms * 1e-3) / 1e12,
+        "fwd_bwd_tflops_3p5x": job_throughput(world, fwd_f + bwd_f, steps, total_ms),
         "pct_of_peak": {"fwd": fwd_f / (fwd_ms * 1e-3) / 1e12 / peak_sus,
                         "fwd_bwd_2p5x": value / world / peak_sus,
                         "fwd_bwd_3p5x": (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12 / peak_sus,

@@ -11,6 +11,22 @@
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
 
+namespace fa {
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing will
+// ever arrive on, through the same routine every pipeline wait uses, with a short
+// limit. The wait gives up, records FA_ERR_TIMEOUT in the status word and the kernel
+// returns normally.
+__global__ void fa_selftest_wait_kernel(long long limit_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_cycles);
+}
+}  // namespace fa
+
 namespace {
 
 constexpr int kVersion = 1;
@@ -360,6 +376,12 @@ int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
   if (st != FA_OK) return st;
   return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype,
                  scratch, stream, kStageAll);
+}
+
+int fa_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles <= 0 || limit_cycles > fa::kWaitLimitCycles) return FA_ERR_INVALID;
+  fa::fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 #ifdef FA_TRACE

@@ -39,6 +39,7 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int,
                               _int, _int, _f32, _int, _vp]),
     "fa_get_device_status": (_int, [_vp]),
+    "fa_selftest_wait_timeout": (_int, [ctypes.c_longlong, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_int]),
     "fa_version": (_int, []),
 }

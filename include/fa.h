@@ -152,6 +152,16 @@ int fa_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O, c
  */
 int fa_get_device_status(void *stream);
 
+/*
+ * Self-test of the device-side failure detection: launches one tiny kernel that waits
+ * on a barrier nothing will complete, with the bounded-wait routine every kernel of
+ * this library uses and a limit of `limit_cycles` SM clock cycles (1 .. 4e9). The
+ * wait gives up and records FA_ERR_TIMEOUT, so the next fa_get_device_status(stream)
+ * returns FA_ERR_TIMEOUT (and clears it); the context stays usable. FA_ERR_INVALID
+ * for a limit out of range.
+ */
+int fa_selftest_wait_timeout(long long limit_cycles, void *stream);
+
 /* Static, human-readable name of a status code. */
 const char *fa_status_string(int status);
 

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
     names = _declared_functions()
     assert names == sorted(["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_status",
                             "fa_status_string", "fa_version", "fa_bwd_preprocess",
-                            "fa_bwd_dkdv", "fa_bwd_dq_convert", "fa_bwd_noalloc"])
+                            "fa_bwd_dkdv", "fa_bwd_dq_convert", "fa_bwd_noalloc",
+                            "fa_selftest_wait_timeout"])
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -117,6 +118,12 @@ def test_fwd_rejects_before_launch(lib, kw, code):
 ])
 def test_bwd_rejects_before_launch(lib, kw, code):
     assert _bwd(lib, **kw) == code
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
+    assert lib.fa_selftest_wait_timeout(-5, None) == fa.FA_ERR_INVALID
+    assert lib.fa_selftest_wait_timeout(10 ** 12, None) == fa.FA_ERR_INVALID
 
 
 def test_binding_raises_without_library(monkeypatch, tmp_path):
