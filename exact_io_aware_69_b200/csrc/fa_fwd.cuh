@@ -68,7 +68,7 @@ struct FwdLayout {
   // for the second row sum
   static constexpr uint32_t kRed = kV + kFwdVStages * kTileBytes;
   static constexpr uint32_t kBar = kRed + 2 * 2 * 2 * 128 * 4;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 20;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 8;
   static constexpr uint32_t kBytes = kAbort + 8 + 1024;  // + alignment slack
@@ -83,10 +83,10 @@ enum : int {
   kBarVEmpty = kBarVFull + kFwdVStages,  // + V stage
   kBarSFull = kBarVEmpty + kFwdVStages,  // + S buffer
   kBarPFull = kBarSFull + 2,             // + S buffer
-  kBarODone = kBarPFull + 2,
-  kFwdNumBars = kBarODone + 1,
+  kBarODone = kBarPFull + 2,            // + (tile & 1): P_j V_j done
+  kFwdNumBars = kBarODone + 2,
 };
-static_assert(kFwdNumBars <= 16, "barrier area");
+static_assert(kFwdNumBars <= 20, "barrier area");
 
 template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(bar(kBarPFull + s), 256);
     }
     mbar_init(bar(kBarODone), 1);
+    mbar_init(bar(kBarODone + 1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                    (jj > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(bar(kBarVEmpty + vs));
-          mma_commit(bar(kBarODone));
+          mma_commit(bar(kBarODone + b));
           FA_TRACE_EVENT(jj, 2);
         }
       }
@@ -304,13 +305,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       l = l * alpha + (a0 + a1);
       l_o = l_o * alpha + (b0 + b1);
       if (threadIdx.x == 0) FA_TRACE_EVENT(j, 5);
-      if (j > 0) {
-        // the previous P V must have landed before O is touched
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone), (j - 1) & 1, abort_flag));
+      // O is touched only when a row's reference moved (rare after the first tiles);
+      // then P_{j-1} V_{j-1} must have landed first. Two alternating barriers make the
+      // skipped waits safe: S_j, complete by now, was issued after P_{j-2} V_{j-2}, so
+      // the barrier of P_{j-1} V_{j-1} is at most one phase away from the one waited.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + ((j - 1) & 1)),
+                                               static_cast<uint32_t>((j - 1) >> 1) & 1, abort_flag));
         if (!ok) continue;
         if (threadIdx.x == 0) FA_TRACE_EVENT(j, 6);
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        {
 #pragma unroll
           for (int c = 0; c < D / 64; ++c) {
             uint32_t o[32];
@@ -329,7 +334,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (threadIdx.x == 0) FA_TRACE_EVENT(j, 7);
       m = m_new;
     }
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarODone), (nkv - 1) & 1, abort_flag));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarODone + ((nkv - 1) & 1)),
+                                                 static_cast<uint32_t>((nkv - 1) >> 1) & 1,
+                                                 abort_flag));
     // both halves' sums: reuse the exchange buffer of parity (nkv & 1), which the pair
     // last used two tiles ago
     red[((nkv & 1) * 2 + half) * 128 + r] = l;
