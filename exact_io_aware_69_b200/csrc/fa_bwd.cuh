@@ -9,8 +9,11 @@
 //   dQ = scale * dS K,   dK = scale * dS^T Q.
 //
 // Three kernels:
-//   fa_bwd_pre_kernel   D = rowsum(dO * (O + O_res)) (fp32; O_res is the forward's
-//                       rounding residual of O, optional), Ls = L * log2(e), dQacc = 0.
+//   fa_bwd_pre_kernel   -D with D = rowsum(dO * (O + O_res)) (fp32; O_res is the
+//                       forward's rounding residual of O, optional), -L * log2(e),
+//                       dQacc = 0. The two row vectors are stored negated so that the
+//                       main kernel forms s * c - L log2(e) and dP - D with packed
+//                       fp32x2 FMA/add and no extra negation.
 //   fa_bwd_main_kernel  one CTA per 128-key tile j of one head: K_j, V_j stay in
 //                       shared memory, the CTA walks the query tiles i that see
 //                       them, accumulates dK_j and dV_j in TMEM, and adds each
@@ -126,8 +129,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (row < rows && part == 0) {
-    Dv[row] = acc;
-    Ls[row] = L[row] * 1.4426950408889634074f;
+    Dv[row] = -acc;
+    Ls[row] = L[row] * -1.4426950408889634074f;
   }
 }
 
@@ -260,19 +263,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t id_sq = idesc_f16_f32(kTile, kTile, BF16, false, false);  // S^T, dP^T
       constexpr uint32_t id_acc = idesc_f16_f32(kTile, D, BF16, false, true);      // dV, dK
       constexpr uint32_t id_dq = idesc_f16_f32(kTile, D, BF16, true, true);        // dQ
-      const uint32_t sk = sbase + Lay::kK, sv = sbase + Lay::kV, sds = sbase + Lay::kDS;
-      const uint32_t sdo = sbase + Lay::kDO;
+      // operand descriptors, built once: K-major views for S^T/dP^T/dK's A, MN-major
+      // views for the B operands of dV/dK/dQ and dQ's A
+      const uint64_t dk_k = sdesc_sw128(sbase + Lay::kK, 16, 1024);
+      const uint64_t dv_k = sdesc_sw128(sbase + Lay::kV, 16, 1024);
+      const uint64_t ddo_k = sdesc_sw128(sbase + Lay::kDO, 16, 1024);
+      const uint64_t dds_k = sdesc_sw128(sbase + Lay::kDS, 16, 1024);
+      const uint64_t dk_mn = sdesc_sw128(sbase + Lay::kK, Lay::kChunkBytes, 1024);
+      const uint64_t ddo_mn = sdesc_sw128(sbase + Lay::kDO, Lay::kChunkBytes, 1024);
+      const uint64_t dds_mn = sdesc_sw128(sbase + Lay::kDS, Lay::kChunkBytes, 1024);
       auto issue_s = [&](int it) -> bool {  // G1: S^T = K_j Q_i^T
         const int st = it & 1;
         if (!mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t sq = sbase + Lay::kQ + st * Lay::kTileBytes;
+        const uint64_t dq = sdesc_sw128(sbase + Lay::kQ + st * Lay::kTileBytes, 16, 1024);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tS, sdesc_sw128(sk + off, 16, 1024), sdesc_sw128(sq + off, 16, 1024),
-                 id_sq, k > 0 ? 1u : 0u);
+          mma_ss(tmem + Lay::tS, sdesc_advance(dk_k, off), sdesc_advance(dq, off), id_sq,
+                 k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbSFull));
         FA_TRACE_EVENT(it, 2);
@@ -284,8 +294,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDP, sdesc_sw128(sv + off, 16, 1024),
-                 sdesc_sw128(sdo + off, 16, 1024), id_sq, k > 0 ? 1u : 0u);
+          mma_ss(tmem + Lay::tDP, sdesc_advance(dv_k, off), sdesc_advance(ddo_k, off), id_sq,
+                 k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbDPFull));
         FA_TRACE_EVENT(it, 4);
@@ -302,8 +312,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8,
-                 sdesc_sw128(sdo + k * 2048, Lay::kChunkBytes, 1024), id_acc,
+          mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8, sdesc_advance(ddo_mn, k * 2048), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar(kBbDOEmpty));  // dO_i has been read for the last time
         FA_TRACE_EVENT(it, 3);
@@ -314,18 +323,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (D != 128 && it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
         tc_fence_after();
         // dK += dS^T Q_i
+        const uint64_t dq_mn = sdesc_sw128(sq, Lay::kChunkBytes, 1024);
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDK, sdesc_sw128(sds + off, 16, 1024),
-                 sdesc_sw128(sq + k * 2048, Lay::kChunkBytes, 1024), id_acc,
+          mma_ss(tmem + Lay::tDK, sdesc_advance(dds_k, off), sdesc_advance(dq_mn, k * 2048), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         }
         // dQ_i = dS K_j   (dS read M-major from the same shared tile)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          mma_ss(tmem + Lay::tDQ, sdesc_sw128(sds + k * 2048, Lay::kChunkBytes, 1024),
-                 sdesc_sw128(sk + k * 2048, Lay::kChunkBytes, 1024), id_dq, k > 0 ? 1u : 0u);
+          mma_ss(tmem + Lay::tDQ, sdesc_advance(dds_mn, k * 2048), sdesc_advance(dk_mn, k * 2048),
+                 id_dq, k > 0 ? 1u : 0u);
         mma_commit(bar(kBbQEmpty + st));
         mma_commit(bar(kBbDSFree));
         mma_commit(bar(kBbDQFull));
@@ -375,15 +384,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       named_bar_sync(1 + quarter, 64);
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 8);
+      const uint64_t c2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int q = c * 32 + e;  // query column within this half
-          float x = ex2_approx(fmaf(p[q], scale_log2, -sL[q]));
-          if (diag && half * 64 + q < r) x = 0.f;
-          p[q] = x;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int q = c * 32 + e4 * 4;  // query column within this half
+          // -L log2(e) of four query columns (a broadcast read)
+          const float4 nl = *reinterpret_cast<const float4*>(sL + q);
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(p[q], p[q + 1]), c2, f2_pack(nl.x, nl.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(p[q + 2], p[q + 3]), c2, f2_pack(nl.z, nl.w)), x2, x3);
+          p[q] = ex2_approx(x0);
+          p[q + 1] = ex2_approx(x1);
+          p[q + 2] = ex2_approx(x2);
+          p[q + 3] = ex2_approx(x3);
+          if (diag) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (half * 64 + q + e < r) p[q + e] = 0.f;
+          }
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) pk[e] = pack2<BF16>(p[c * 32 + 2 * e], p[c * 32 + 2 * e + 1]);
@@ -408,12 +429,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           uint32_t ds[4];
+          // -D of eight query columns (broadcast reads)
+          const float4 nd0 = *reinterpret_cast<const float4*>(sD + c * 32 + 8 * u);
+          const float4 nd1 = *reinterpret_cast<const float4*>(sD + c * 32 + 8 * u + 4);
+          const float ndv[8] = {nd0.x, nd0.y, nd0.z, nd0.w, nd1.x, nd1.y, nd1.z, nd1.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int k = 8 * u + 2 * e;  // column within this 32-column chunk
             const int q = c * 32 + k;
-            const float a = p[q] * (__uint_as_float(dr[k]) - sD[q]);
-            const float b = p[q + 1] * (__uint_as_float(dr[k + 1]) - sD[q + 1]);
+            // dS = P (dP - D), two columns per packed fp32x2 add and multiply
+            float a, b;
+            f2_unpack(f2_mul(f2_pack(p[q], p[q + 1]),
+                             f2_add(f2_pack(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])),
+                                    f2_pack(ndv[2 * e], ndv[2 * e + 1]))),
+                      a, b);
             ds[e] = pack2<BF16>(a, b);
           }
           const int unit = (c * 4 + u) ^ sw;
@@ -466,21 +495,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t* stage_row = smem + Lay::kStage + qr * 128;
     const int sw = qr & 7;
     for (int it = 0; it < niter; ++it) {
-      // the four drain warps decide together, so that all of them meet every named barrier
-      if (!named_bar_and(5, 128,
-                         mbar_wait(bar(kBbDQFull), static_cast<uint32_t>(it & 1), abort_flag)))
-        break;
-      if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
-      tc_fence_after();
+      // Each warp frees its TMEM lanes as soon as dQ_i is there (the next dP^T MMA
+      // waits for that); the four warps agree before touching the shared staging
+      // buffer, so that all of them meet every named barrier below.
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar(kBbDQFull),
+                                                         static_cast<uint32_t>(it & 1), abort_flag));
       uint32_t v[D];
+      if (got) {
+        if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
+        tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
-      tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
-      tc_fence_before();
-      mbar_arrive(bar(kBbDQEmpty));
-      if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
+        for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
+        tc_fence_before();
+        mbar_arrive(bar(kBbDQEmpty));
+        if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
+      }
+      if (!named_bar_and(5, 128, got)) break;
       const int row = static_cast<int>(head_row) + (i_begin + it) * kTile;
 #pragma unroll
       for (int rnd = 0; rnd < D / 64; ++rnd) {

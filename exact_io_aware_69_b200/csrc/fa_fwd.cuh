@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_f16_f32(kTile, kTile, BF16, false, false);
       constexpr uint32_t idesc_o = idesc_f16_f32(kTile, D, BF16, false, true);
-      const uint32_t sq = sbase + Lay::kQ;
+      const uint64_t dq = sdesc_sw128(sbase + Lay::kQ, 16, 1024);
       bool ok = mbar_wait(bar(kBarQFull), 0, abort_flag);
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {
@@ -193,13 +193,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t kuse = static_cast<uint32_t>(j / kFwdKStages);
           if (!mbar_wait(bar(kBarKFull + ks), kuse & 1, abort_flag)) break;
           tc_fence_after();
-          const uint32_t sk = sbase + Lay::kK + ks * Lay::kTileBytes;
+          const uint64_t dk = sdesc_sw128(sbase + Lay::kK + ks * Lay::kTileBytes, 16, 1024);
           const uint32_t d_s = tmem + (j & 1) * 128;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-            mma_ss(d_s, sdesc_sw128(sq + off, 16, 1024), sdesc_sw128(sk + off, 16, 1024), idesc_s,
-                   k > 0 ? 1u : 0u);
+            mma_ss(d_s, sdesc_advance(dq, off), sdesc_advance(dk, off), idesc_s, k > 0 ? 1u : 0u);
           }
           mma_commit(bar(kBarKEmpty + ks));
           mma_commit(bar(kBarSFull + (j & 1)));
@@ -215,14 +214,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                          abort_flag))
             break;
           tc_fence_after();
-          const uint32_t sv = sbase + Lay::kV + vs * Lay::kTileBytes;
+          const uint64_t dv = sdesc_sw128(sbase + Lay::kV + vs * Lay::kTileBytes,
+                                          Lay::kChunkBytes, 1024);
           const uint32_t a_p = tmem + b * 128;  // P packed in the first 64 columns
           const uint32_t d_o = tmem + 256;
 #pragma unroll
-          for (int k = 0; k < kTile / 16; ++k) {
-            mma_ts(d_o, a_p + k * 8, sdesc_sw128(sv + k * 2048, Lay::kChunkBytes, 1024), idesc_o,
+          for (int k = 0; k < kTile / 16; ++k)
+            mma_ts(d_o, a_p + k * 8, sdesc_advance(dv, k * 2048), idesc_o,
                    (jj > 0 || k > 0) ? 1u : 0u);
-          }
           mma_commit(bar(kBarVEmpty + vs));
           mma_commit(bar(kBarODone + b));
           FA_TRACE_EVENT(jj, 2);

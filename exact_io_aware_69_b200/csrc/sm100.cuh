@@ -233,6 +233,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// The same descriptor `bytes` further on in shared memory: the start address is the
+// low 14-bit field (address >> 4), and every shared address here is below 2^18, so a
+// plain add never carries out of it. Lets an MMA loop build each operand's descriptor
+// once and step it with immediate adds.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma.kind::f16 with an fp32 accumulator:
 // D format f32 (bits 4-5 = 1), A/B format bf16 = 1 or f16 = 0 (bits 7-9, 10-12),
 // A/B major (bit 15, 16: 0 = K-major, 1 = MN-major), N >> 3 (bits 17-22),
