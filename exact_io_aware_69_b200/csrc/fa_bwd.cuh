@@ -500,33 +500,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // buffer, so that all of them meet every named barrier below.
       const bool got = __all_sync(0xffffffffu, mbar_wait(bar(kBbDQFull),
                                                          static_cast<uint32_t>(it & 1), abort_flag));
-      uint32_t v[D];
-      if (got) {
-        if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
-        tc_fence_before();
-        mbar_arrive(bar(kBbDQEmpty));
-        if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
-      }
-      if (!named_bar_and(5, 128, got)) break;
+      // Two rounds of 64 columns (64 registers each, no spills): the first round is
+      // staged and handed to the TMA unit before the second leaves TMEM; the columns
+      // are released after the second.
       const int row = static_cast<int>(head_row) + (i_begin + it) * kTile;
+      bool all_ok = true;
 #pragma unroll
       for (int rnd = 0; rnd < D / 64; ++rnd) {
-        if (leader) bulk_wait_read_all();  // previous round's boxes have been read
-        named_bar_sync(5, 128);
+        uint32_t v[64];
+        if (got) {
+          if (rnd == 0 && warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
+          tc_fence_after();
+          tmem_ld32(lane_base + Lay::tDQ + rnd * 64, v);
+          tmem_ld32(lane_base + Lay::tDQ + rnd * 64 + 32, v + 32);
+          tmem_wait_ld();
+          reg_fence32(v);
+          reg_fence32(v + 32);
+          if (rnd == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar(kBbDQEmpty));
+            if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
+          }
+        }
+        // all four warps agree (and the previous round's boxes have been read)
+        // before anyone writes the staging buffer
+        if (leader) bulk_wait_read_all();
+        all_ok = named_bar_and(5, 128, got);
+        if (!all_ok) break;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int box = 2 * rnd + h;  // columns 32 box .. 32 box + 31
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(stage_row + h * Lay::kChunkBytes + ((u ^ sw) * 16)) =
-                make_uint4(v[32 * box + 4 * u], v[32 * box + 4 * u + 1],
-                           v[32 * box + 4 * u + 2], v[32 * box + 4 * u + 3]);
+                make_uint4(v[32 * h + 4 * u], v[32 * h + 4 * u + 1], v[32 * h + 4 * u + 2],
+                           v[32 * h + 4 * u + 3]);
         }
         fence_async_smem();
         named_bar_sync(5, 128);
@@ -537,6 +544,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           bulk_commit();
         }
       }
+      if (!all_ok) break;
       if (leader) FA_TRACE_EVENT(it, 14);
     }
     if (leader) bulk_wait_all();  // every reduce-add has landed before the CTA exits
