@@ -164,6 +164,12 @@ int launch_bwd(const BwdArgs& a, int stages) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return FA_ERR_CUDA;
+    // The kernel moves registers between warpgroups (setmaxnreg); its split adds up to
+    // exactly 128 registers per thread at launch. Launched with fewer, the increase
+    // would wait for registers that never come back, so refuse instead.
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FA_ERR_CUDA;
+    if (attr.numRegs != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
     const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.N / fa::kTile);
     kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
         *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
@@ -392,6 +398,11 @@ int fa_trace_attach(void* buf, const int* ctas) {
   if (cudaMemcpyToSymbol(fa::g_fa_trace_cta, ctas, sizeof(int) * fa::kTraceSlots) != cudaSuccess)
     return FA_ERR_CUDA;
   return FA_OK;
+}
+// Trace builds only: a device buffer of 8 uint64 per CTA for the per-CTA life log.
+int fa_trace_cta_log(void* buf) {
+  return cudaMemcpyToSymbol(fa::g_fa_cta_log, &buf, sizeof(void*)) == cudaSuccess ? FA_OK
+                                                                                : FA_ERR_CUDA;
 }
 #endif
 

@@ -20,8 +20,8 @@
 //                       dQ_i partial into the fp32 accumulator with TMA reduce-adds.
 //   fa_bwd_dq_kernel    dQ = dtype(scale * dQacc).
 //
-// Main-kernel warp roles (448 threads; 14 warps keep 4 or fewer per SM sub-partition,
-// which leaves each thread up to 128 registers):
+// Main-kernel warp roles (512 threads = 4 warpgroups; at launch every thread may
+// hold 128 registers, then warpgroup 3 hands registers to warpgroup 2 with setmaxnreg):
 //   warps 0-7  compute, in pairs: warps w and w+4 share TMEM lane quarter w % 4, so
 //              thread r of the pair owns key row r = 32 (w % 4) + lane; warp w < 4
 //              takes query columns 0-63, warp w+4 columns 64-127 (no row reduction
@@ -29,25 +29,39 @@
 //              dS^T from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to shared
 //              memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
 //              dK_j / dV_j epilogue, each warp of the pair writing half the columns.
-//   warp 8     TMA producer: K_j, V_j once; Q_i, Ls_i, D_i into a 2-stage ring; dO_i
+//   warps 8-11 dQ drain (200 registers each): thread owns query row (warp % 4) * 32 +
+//              lane; takes the whole dQ_i row out of TMEM at once, so that the
+//              columns are free again after one round of loads, then stages it in
+//              shared memory and has the TMA unit add it into the fp32 accumulator
+//              (cp.reduce.async.bulk.tensor).
+//   warp 12    TMA producer: K_j, V_j once; Q_i, Ls_i, D_i into a 2-stage ring; dO_i
 //              into a single buffer (its last reader, the dV MMA, finishes well
 //              before the next dP^T MMA needs the next tile).
-//   warp 9     MMA issuer (and TMEM owner), per query tile:
+//   warp 13    MMA issuer (and TMEM owner), per query tile:
 //                S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (SMEM x SMEM)
 //                dV += P^T dO_i                              (P^T from TMEM)
 //                dK += dS^T Q_i, dQ_i = dS K_j                (dS from SMEM)
-//   warps 10-13 dQ drain: thread owns query row (warp % 4) * 32 + lane; copies the
-//              dQ_i tile out of TMEM, stages it in shared memory and has the TMA unit
-//              add it into the fp32 accumulator (cp.reduce.async.bulk.tensor).
+//   warps 14-15 idle (they complete warpgroup 3, which runs on 56 registers).
 #pragma once
 
 #include "sm100.cuh"
 
 namespace fa {
 
-constexpr int kBwdThreads = 448;
-constexpr int kBwdProducerWarp = 8;
-constexpr int kBwdMmaWarp = 9;
+constexpr int kBwdThreads = 512;
+constexpr int kBwdDrainWarp0 = 8;  // warpgroup 2
+constexpr int kBwdProducerWarp = 12;
+constexpr int kBwdMmaWarp = 13;
+// Registers per thread after the split: 2 x 128 (compute) + 200 (drain) + 56 = 4 x 128,
+// the budget of one sub-partition (one warp of each warpgroup) at launch, when every
+// thread holds kBwdLaunchRegs (the most 512 threads can have; the host checks that
+// the compiled kernel uses exactly that many).
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kBwdDrainRegs = 200;
+constexpr int kBwdSmallRegs = 56;
+static_assert(kBwdThreads * kBwdLaunchRegs == 65536, "launch register budget");
+static_assert(2 * kBwdLaunchRegs + kBwdDrainRegs + kBwdSmallRegs == 4 * kBwdLaunchRegs,
+              "register split");
 
 template <int D>
 struct BwdLayout {
@@ -174,6 +188,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_base + pad;
 
+  FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ntiles = N / kTile;
@@ -211,11 +226,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  FA_TRACE_BEGIN();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
 
   if (warp == kBwdProducerWarp) {
     // ------------------------------------------------------------ TMA producer
+    setmaxnreg_dec<kBwdSmallRegs>();  // each role of warpgroup 3 gives registers back
     if (lane == 0) {
       tma_prefetch(&tmQ);
       tma_prefetch(&tmK);
@@ -252,6 +269,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- MMA issuer
+    setmaxnreg_dec<kBwdSmallRegs>();
     // Software-pipelined over the query tiles: with G1 = S^T, G2 = dP^T, G3 = dV,
     // G4 = dK, G5 = dQ, the issue order is
     //   G1(0) G2(0) | G3(0) G1(1) G4(0) G5(0) G2(1) | G3(1) G1(2) G4(1) G5(1) G2(2) | ...
@@ -281,7 +299,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tS, sdesc_advance(dk_k, off), sdesc_advance(dq, off), id_sq,
+          mma_ss(tmem + Lay::tS, sdesc_step(dk_k, off), sdesc_step(dq, off), id_sq,
                  k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbSFull));
@@ -294,7 +312,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDP, sdesc_advance(dv_k, off), sdesc_advance(ddo_k, off), id_sq,
+          mma_ss(tmem + Lay::tDP, sdesc_step(dv_k, off), sdesc_step(ddo_k, off), id_sq,
                  k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbDPFull));
@@ -312,7 +330,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8, sdesc_advance(ddo_mn, k * 2048), id_acc,
+          mma_ts(tmem + Lay::tDV, tmem + Lay::tS + k * 8, sdesc_step(ddo_mn, k * 2048), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         mma_commit(bar(kBbDOEmpty));  // dO_i has been read for the last time
         FA_TRACE_EVENT(it, 3);
@@ -327,13 +345,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
           const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDK, sdesc_advance(dds_k, off), sdesc_advance(dq_mn, k * 2048), id_acc,
+          mma_ss(tmem + Lay::tDK, sdesc_step(dds_k, off), sdesc_step(dq_mn, k * 2048), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         }
         // dQ_i = dS K_j   (dS read M-major from the same shared tile)
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k)
-          mma_ss(tmem + Lay::tDQ, sdesc_advance(dds_mn, k * 2048), sdesc_advance(dk_mn, k * 2048),
+          mma_ss(tmem + Lay::tDQ, sdesc_step(dds_mn, k * 2048), sdesc_step(dk_mn, k * 2048),
                  id_dq, k > 0 ? 1u : 0u);
         mma_commit(bar(kBbQEmpty + st));
         mma_commit(bar(kBbDSFree));
@@ -480,8 +498,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < kBwdDrainWarp0 + 4) {
     // ---------------------------------------------------------------- dQ drain
+    setmaxnreg_inc<kBwdDrainRegs>();
     // dQ_i leaves TMEM into registers (then the MMA warp may reuse the columns), is
     // staged in shared memory in the 128-byte-swizzled layout of a 128-row x 32-column
     // fp32 box, and is added into the fp32 accumulator by TMA reduce-adds that one
@@ -490,7 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quarter = warp & 3;
     const int qr = quarter * 32 + lane;  // query row within tile i
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const bool leader = (warp == 10 && lane == 0);
+    const bool leader = (warp == kBwdDrainWarp0 && lane == 0);
     const uint32_t stage = sbase + Lay::kStage;
     uint8_t* stage_row = smem + Lay::kStage + qr * 128;
     const int sw = qr & 7;
@@ -500,40 +519,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // buffer, so that all of them meet every named barrier below.
       const bool got = __all_sync(0xffffffffu, mbar_wait(bar(kBbDQFull),
                                                          static_cast<uint32_t>(it & 1), abort_flag));
-      // Two rounds of 64 columns (64 registers each, no spills): the first round is
-      // staged and handed to the TMA unit before the second leaves TMEM; the columns
-      // are released after the second.
+      uint32_t v[D];
+      if (got) {
+        if (leader) FA_TRACE_EVENT(it, 12);
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + Lay::tDQ + c * 32, v + c * 32);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) reg_fence32(v + c * 32);
+        tc_fence_before();
+        mbar_arrive(bar(kBbDQEmpty));
+        if (leader) FA_TRACE_EVENT(it, 13);
+      }
+      if (!named_bar_and(5, 128, got)) break;
       const int row = static_cast<int>(head_row) + (i_begin + it) * kTile;
-      bool all_ok = true;
 #pragma unroll
       for (int rnd = 0; rnd < D / 64; ++rnd) {
-        uint32_t v[64];
-        if (got) {
-          if (rnd == 0 && warp == 10 && lane == 0) FA_TRACE_EVENT(it, 12);
-          tc_fence_after();
-          tmem_ld32(lane_base + Lay::tDQ + rnd * 64, v);
-          tmem_ld32(lane_base + Lay::tDQ + rnd * 64 + 32, v + 32);
-          tmem_wait_ld();
-          reg_fence32(v);
-          reg_fence32(v + 32);
-          if (rnd == D / 64 - 1) {
-            tc_fence_before();
-            mbar_arrive(bar(kBbDQEmpty));
-            if (warp == 10 && lane == 0) FA_TRACE_EVENT(it, 13);
-          }
-        }
-        // all four warps agree (and the previous round's boxes have been read)
-        // before anyone writes the staging buffer
-        if (leader) bulk_wait_read_all();
-        all_ok = named_bar_and(5, 128, got);
-        if (!all_ok) break;
+        if (leader) bulk_wait_read_all();  // previous round's boxes have been read
+        named_bar_sync(5, 128);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          const int box = 2 * rnd + h;  // columns 32 box .. 32 box + 31
 #pragma unroll
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(stage_row + h * Lay::kChunkBytes + ((u ^ sw) * 16)) =
-                make_uint4(v[32 * h + 4 * u], v[32 * h + 4 * u + 1], v[32 * h + 4 * u + 2],
-                           v[32 * h + 4 * u + 3]);
+                make_uint4(v[32 * box + 4 * u], v[32 * box + 4 * u + 1],
+                           v[32 * box + 4 * u + 2], v[32 * box + 4 * u + 3]);
         }
         fence_async_smem();
         named_bar_sync(5, 128);
@@ -544,10 +556,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           bulk_commit();
         }
       }
-      if (!all_ok) break;
       if (leader) FA_TRACE_EVENT(it, 14);
     }
     if (leader) bulk_wait_all();  // every reduce-add has landed before the CTA exits
+  } else {
+    setmaxnreg_dec<kBwdSmallRegs>();  // warps 14-15: no role
   }
 
   tc_fence_before();
@@ -557,6 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  FA_TRACE_CTA(1);
 }
 
 }  // namespace fa

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_base + pad;
 
+  FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ntiles = N / kTile;
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  FA_TRACE_BEGIN();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
 
@@ -385,6 +387,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  FA_TRACE_CTA(1);
 }
 
 }  // namespace fa

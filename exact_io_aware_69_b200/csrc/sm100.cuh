@@ -35,15 +35,41 @@ constexpr int kTraceEvents = 16;
 #ifdef FA_TRACE
 __device__ unsigned long long* g_fa_trace = nullptr;
 __device__ int g_fa_trace_cta[kTraceSlots] = {-1, -1, -1, -1};
-__device__ __forceinline__ void trace_event(int it, int ev) {
-  if (g_fa_trace == nullptr || it < 0 || it >= kTraceIters) return;
+// This CTA's slot in the trace buffer, or null; looked up once per thread so that an
+// event costs one compare and one store.
+__device__ __forceinline__ unsigned long long* trace_begin() {
+  if (g_fa_trace == nullptr) return nullptr;
 #pragma unroll
   for (int s = 0; s < kTraceSlots; ++s)
     if (g_fa_trace_cta[s] == static_cast<int>(blockIdx.x))
-      g_fa_trace[(s * kTraceIters + it) * kTraceEvents + ev] = clock64();
+      return g_fa_trace + s * kTraceIters * kTraceEvents;
+  return nullptr;
 }
-#define FA_TRACE_EVENT(it, ev) ::fa::trace_event((it), (ev))
+#define FA_TRACE_BEGIN() unsigned long long* const fa_trace_slot = ::fa::trace_begin()
+// Every CTA's life: [cta][8] = start clock, end clock, SM id, start and end global
+// time (ns). Thread 0 records its own start and end.
+__device__ unsigned long long* g_fa_cta_log = nullptr;
+__device__ __forceinline__ void trace_cta(int end) {
+  unsigned long long* log = g_fa_cta_log;
+  if (log == nullptr || threadIdx.x != 0) return;
+  unsigned long long ns;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(ns));
+  uint32_t smid;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+  log += static_cast<size_t>(blockIdx.x) * 8;
+  log[end] = clock64();
+  log[3 + end] = ns;
+  if (!end) log[2] = smid;
+}
+#define FA_TRACE_CTA(end) ::fa::trace_cta(end)
+#define FA_TRACE_EVENT(it, ev)                                                          \
+  do {                                                                                  \
+    if (fa_trace_slot != nullptr && static_cast<unsigned>(it) < ::fa::kTraceIters)      \
+      fa_trace_slot[(it) * ::fa::kTraceEvents + (ev)] = clock64();                      \
+  } while (0)
 #else
+#define FA_TRACE_BEGIN() ((void)0)
+#define FA_TRACE_CTA(end) ((void)0)
 #define FA_TRACE_EVENT(it, ev) ((void)0)
 #endif
 
@@ -240,6 +266,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 __device__ __forceinline__ uint64_t sdesc_advance(uint64_t desc, uint32_t bytes) {
   return desc + static_cast<uint64_t>(bytes >> 4);
 }
+// The same step, formed where the MMA is issued: an MMA loop whose operand views are
+// all loop-invariant would otherwise keep every stepped descriptor in registers
+// (two per view per step), which a register-lean issuing warp cannot afford.
+__device__ __forceinline__ uint64_t sdesc_step(uint64_t desc, uint32_t bytes) {
+  uint64_t out;
+  asm volatile("add.u64 %0, %1, %2;" : "=l"(out) : "l"(desc), "l"(static_cast<uint64_t>(bytes >> 4)));
+  return out;
+}
 
 // Instruction descriptor of tcgen05.mma.kind::f16 with an fp32 accumulator:
 // D format f32 (bits 4-5 = 1), A/B format bf16 = 1 or f16 = 0 (bits 7-9, 10-12),
@@ -287,6 +321,17 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 
 // Named barrier that also ANDs a predicate over its `count` threads: every thread gets
 // true only if all passed true (a group-wide vote, e.g. on whether a wait succeeded).
+// Per-warpgroup register budget (all four warps of a warpgroup execute it together).
+// An increase waits until other warpgroups' decreases have returned enough registers
+// to the pool the CTA was launched with.
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
 __device__ __forceinline__ bool named_bar_and(int id, int count, bool v) {
   uint32_t r;
   asm volatile(
