@@ -103,8 +103,9 @@ int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty)
 }
 
 template <int D, bool CAUSAL, bool BF16>
-int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, void* O,
-               void* O_res, float* L, int BH, int N, float scale, cudaStream_t stream) {
+int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+               const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int BH,
+               int N, float scale, cudaStream_t stream) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, BF16>;
   // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
   // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
@@ -113,8 +114,7 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
       cudaSuccess)
     return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, static_cast<uint16_t*>(O),
-                                                 static_cast<uint16_t*>(O_res), L, N,
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, N,
                                                  scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -269,12 +269,13 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, fl
       !aligned16(O_res))
     return FA_ERR_INVALID;
   const long rows = static_cast<long>(B) * H * N;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to, tr;
   if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
-      !make_tmap(&tv, V, rows, d, dtype))
+      !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&to, O, rows, d, dtype) ||
+      !make_tmap(&tr, O_res != nullptr ? O_res : O, rows, d, dtype))
     return FA_ERR_CUDA;
-  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, O, O_res, L, B * H, N, scale,
-                          static_cast<cudaStream_t>(stream));
+  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, B * H, N,
+                          scale, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {

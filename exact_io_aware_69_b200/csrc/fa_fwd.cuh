@@ -91,9 +91,9 @@ static_assert(kFwdNumBars <= 20, "barrier area");
 template <int D, bool CAUSAL, bool BF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, uint16_t* __restrict__ O,
-                  uint16_t* __restrict__ O_res, float* __restrict__ Lse, int N,
-                  float scale_log2) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const __grid_constant__ CUtensorMap tmOres, bool has_res,
+                  float* __restrict__ Lse, int N, float scale_log2) {
   using Lay = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -345,19 +345,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     named_bar_sync(pair_bar, 64);
     const float l_row = l + red[((nkv & 1) * 2 + (half ^ 1)) * 128 + r];
     const float l_o_row = l_o + red[((nkv & 1) * 2 + (half ^ 1)) * 128 + r + 512];
+    // O and its rounding residual go out through shared memory and TMA stores (whole
+    // 128-byte lines), staged in the K ring, which the finished last S MMA has freed:
+    // the 128-row x 64-column chunk c of O at kK + c * kChunkBytes, of O_res one tile
+    // further on, each in the 128-byte-swizzled layout of the tensor maps.
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.f / l_o_row;
-      const size_t obase = static_cast<size_t>(row0 + r) * D + half * (D / 2);
+      const uint32_t st_o = sbase + Lay::kK;
+      const uint32_t st_r = st_o + Lay::kTileBytes;
+      const int sw = r & 7;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
         tmem_ld32(lane_base + o_cols + c * 32, o);
         tmem_wait_ld();
         reg_fence32(o);
-        uint4 hi[4], lo[4];
-        uint32_t* hw = reinterpret_cast<uint32_t*>(hi);
-        uint32_t* lw = reinterpret_cast<uint32_t*>(lo);
+        uint32_t hw[16], lw[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float x0 = __uint_as_float(o[2 * e]) * inv_l;
@@ -367,16 +371,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           unpack2<BF16>(hw[e], h0, h1);
           lw[e] = pack2<BF16>(x0 - h0, x1 - h1);  // exact difference, then rounded
         }
-        uint4* dst = reinterpret_cast<uint4*>(O + obase + c * 32);
+        // this thread's 32 columns: half * D/2 + 32 c .. +31
+        const int col = half * (D / 2) + c * 32;
+        const uint32_t chunk = static_cast<uint32_t>(col / 64) * Lay::kChunkBytes + r * 128;
+        const int u0 = (col % 64) / 8;  // first 16-byte unit within the 128-byte row
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = hi[e];
-        if (O_res != nullptr) {
-          uint4* dres = reinterpret_cast<uint4*>(O_res + obase + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dres[e] = lo[e];
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t off = chunk + static_cast<uint32_t>(((u0 + u) ^ sw) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(st_o + off),
+                       "r"(hw[4 * u]), "r"(hw[4 * u + 1]), "r"(hw[4 * u + 2]), "r"(hw[4 * u + 3])
+                       : "memory");
+          if (has_res)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(st_r + off),
+                         "r"(lw[4 * u]), "r"(lw[4 * u + 1]), "r"(lw[4 * u + 2]),
+                         "r"(lw[4 * u + 3])
+                         : "memory");
         }
       }
+      fence_async_smem();
       if (half == 0) Lse[row0 + r] = (m + log2f(l_row)) * 0.69314718055994530942f;
+    }
+    // all 256 softmax threads have staged their part (or all gave up together)
+    if (named_bar_and(5, 256, ok) && threadIdx.x == 0) {
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_store_2d(&tmO, sbase + Lay::kK + c * Lay::kChunkBytes, c * 64, row0);
+        if (has_res)
+          tma_store_2d(&tmOres, sbase + Lay::kK + Lay::kTileBytes + c * Lay::kChunkBytes, c * 64,
+                       row0);
+      }
+      bulk_commit();
+      bulk_wait_read_all();  // shared memory is read before the CTA releases it
     }
   }
 
