@@ -106,14 +106,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Waits until the barrier phase with `parity` has completed. Gives up (returns false)
 // when another role of the CTA raised `abort`, or after kWaitLimitCycles; in the
 // latter case it raises `abort` itself and records FA_ERR_TIMEOUT in g_fa_status.
+// Only a wait that has already lasted kAbortPollCycles reads the shared abort flag:
+// ordinary waits are short, and a load per spin would compete for shared-memory
+// bandwidth with the tensor cores' operand reads.
+constexpr long long kAbortPollCycles = 200000;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           long long limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    const long long waited = clock64() - t0;
+    if (waited < kAbortPollCycles && waited <= limit_cycles) continue;
     if (*abort) return false;
-    if (clock64() - t0 > limit_cycles) {
+    if (waited > limit_cycles) {
       *abort = 1;
       atomicExch(&g_fa_status, kStatusTimeout);
       return false;
