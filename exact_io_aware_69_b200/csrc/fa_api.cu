@@ -51,35 +51,33 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows, d] row-major 16-bit tensor, box of 64 columns x 128 rows, 128-byte swizzle.
-bool make_tmap(CUtensorMap* map, const void* ptr, long rows, int d, int dtype) {
+// [BH][N][d] row-major tensor seen in three dimensions (column, row within a head,
+// head), so that a 128-row box reaching past a head's N reads zeros and writes
+// nothing there. 16-bit: box of 64 columns x 128 rows; fp32 (the dQ accumulator,
+// target of TMA reduce-adds): 32 columns (128 bytes) x 128 rows. 128-byte swizzle.
+bool make_tmap3(CUtensorMap* map, const void* ptr, int BH, int N, int d,
+                CUtensorMapDataType type, int esize) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   2, const_cast<void*>(ptr), dims, strides, box, estr,
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
+                           static_cast<cuuint64_t>(N) * d * esize};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-
-// [rows, d] row-major fp32 tensor, box of 32 columns (128 bytes) x 128 rows,
-// 128-byte swizzle: the dQ accumulator, target of TMA reduce-adds.
-bool make_tmap_f32(CUtensorMap* map, const void* ptr, long rows, int d) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 4};
-  cuuint32_t box[2] = {32, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+bool make_tmap(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype) {
+  return make_tmap3(map, ptr, BH, N, d,
+                    dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                     : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    2);
+}
+bool make_tmap_f32(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+  return make_tmap3(map, ptr, BH, N, d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -96,9 +94,9 @@ int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty)
     *empty = true;
     return FA_OK;
   }
-  if (N % fa::kTile != 0) return FA_ERR_UNSUPPORTED;
-  // TMA coordinates and grid indices are 32-bit
-  if (static_cast<long long>(B) * H * N >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  // TMA coordinates and grid indices are 32-bit (rows counted with N padded to 128)
+  if (static_cast<long long>(B) * H * ((N + fa::kTile - 1) / fa::kTile * fa::kTile) >= (1LL << 31))
+    return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -113,7 +111,8 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(BH) * static_cast<unsigned>(N / fa::kTile);
+  const unsigned grid =
+      static_cast<unsigned>(BH) * static_cast<unsigned>((N + fa::kTile - 1) / fa::kTile);
   kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, N,
                                                  scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -141,19 +140,22 @@ struct BwdArgs {
 
 enum { kStagePre = 1, kStageMain = 2, kStageDq = 4, kStageAll = 7 };
 
-// Workspace: D [rows] fp32, Ls [rows] fp32, dQ accumulator [rows][d] fp32.
+// Workspace: D and Ls as [BH][n_pad] fp32 (n_pad = N rounded up to 128, so that every
+// query tile reads whole 512-byte rows), then the dQ accumulator [BH][N][d] fp32.
 template <int D, bool CAUSAL, bool BF16>
 int launch_bwd(const BwdArgs& a, int stages) {
   const long rows = static_cast<long>(a.BH) * a.N;
+  const int n_pad = (a.N + fa::kTile - 1) / fa::kTile * fa::kTile;
+  const long prows = static_cast<long>(a.BH) * n_pad;
   float* Dv = static_cast<float*>(a.workspace);
-  float* Ls = Dv + rows;
-  float* dq_acc = Ls + rows;
+  float* Ls = Dv + prows;
+  float* dq_acc = Ls + prows;
   if (stages & kStagePre) {
-    const long threads = rows * (D / 8);
+    const long threads = prows * (D / 8);
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
         static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.O_res),
-        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, rows);
+        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, a.N, n_pad, prows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stages & kStageMain) {
@@ -170,7 +172,7 @@ int launch_bwd(const BwdArgs& a, int stages) {
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FA_ERR_CUDA;
     if (attr.numRegs != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
-    const unsigned grid = static_cast<unsigned>(a.BH) * static_cast<unsigned>(a.N / fa::kTile);
+    const unsigned grid = static_cast<unsigned>(prows / fa::kTile);
     kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
         *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
         static_cast<uint16_t*>(a.dV), a.N, a.scale, a.scale * 1.4426950408889634074f,
@@ -268,11 +270,11 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, fl
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L) ||
       !aligned16(O_res))
     return FA_ERR_INVALID;
-  const long rows = static_cast<long>(B) * H * N;
+  const int BH = B * H;
   CUtensorMap tq, tk, tv, to, tr;
-  if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
-      !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&to, O, rows, d, dtype) ||
-      !make_tmap(&tr, O_res != nullptr ? O_res : O, rows, d, dtype))
+  if (!make_tmap(&tq, Q, BH, N, d, dtype) || !make_tmap(&tk, K, BH, N, d, dtype) ||
+      !make_tmap(&tv, V, BH, N, d, dtype) || !make_tmap(&to, O, BH, N, d, dtype) ||
+      !make_tmap(&tr, O_res != nullptr ? O_res : O, BH, N, d, dtype))
     return FA_ERR_CUDA;
   return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, B * H, N,
                           scale, static_cast<cudaStream_t>(stream));
@@ -282,9 +284,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   if (B < 0 || H < 0 || N < 0 || d < 0) return static_cast<size_t>(-1);
   const size_t rows = static_cast<size_t>(B) * H * N;
   if (rows == 0) return 0;
-  // D and Ls (fp32 per row), then the fp32 dQ accumulator; every part 256-aligned
-  // because rows is a multiple of 128 for every supported shape.
-  return rows * 4 * 2 + rows * static_cast<size_t>(d) * 4;
+  // D and Ls (fp32 per row, N padded to a multiple of 128 per head), then the fp32 dQ
+  // accumulator; its start is 1024-byte aligned because the padded row count is a
+  // multiple of 128.
+  const size_t n_pad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return static_cast<size_t>(B) * H * n_pad * 4 * 2 + rows * static_cast<size_t>(d) * 4;
 }
 
 // Validation shared by fa_bwd and its stages; the pointers a stage does not use may
@@ -301,13 +305,14 @@ static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* 
 static int bwd_run(const void* Q, const void* K, const void* V, const void* O,
             const void* O_res, const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
             int causal, float scale, int dtype, void* workspace, void* stream, int stages) {
-  const long rows = static_cast<long>(B) * H * N;
+  const int BH = B * H;
+  const long prows = static_cast<long>(BH) * ((N + fa::kTile - 1) / fa::kTile * fa::kTile);
   CUtensorMap tq, tk, tv, tdo, tdq;
   if (stages & kStageMain) {
-    const float* dq_acc = static_cast<const float*>(workspace) + 2 * rows;
-    if (!make_tmap(&tq, Q, rows, d, dtype) || !make_tmap(&tk, K, rows, d, dtype) ||
-        !make_tmap(&tv, V, rows, d, dtype) || !make_tmap(&tdo, dO, rows, d, dtype) ||
-        !make_tmap_f32(&tdq, dq_acc, rows, d))
+    const float* dq_acc = static_cast<const float*>(workspace) + 2 * prows;
+    if (!make_tmap(&tq, Q, BH, N, d, dtype) || !make_tmap(&tk, K, BH, N, d, dtype) ||
+        !make_tmap(&tv, V, BH, N, d, dtype) || !make_tmap(&tdo, dO, BH, N, d, dtype) ||
+        !make_tmap_f32(&tdq, dq_acc, BH, N, d))
       return FA_ERR_CUDA;
   }
   BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, O, O_res, dO, L, dQ, dK, dV, B * H, N, scale, workspace,

@@ -107,19 +107,25 @@ enum : int {
 };
 
 // ------------------------------------------------------------------ preprocess
-// One group of D/8 threads per row: 8 elements (16 bytes) per thread.
+// One group of D/8 threads per row: 8 elements (16 bytes) per thread. Rows are walked
+// in the padded per-head layout of Dv and Ls (n_pad = 128 * ceil(N / 128) rows per
+// head); a padded row gets D = 0 and -L log2(e) = -inf, so that its p is exactly 0.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
     fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ O_res,
                       const uint16_t* __restrict__ dO, const float* __restrict__ L,
-                      float* __restrict__ Dv,
-                      float* __restrict__ Ls, float* __restrict__ dq_acc, long rows) {
+                      float* __restrict__ Dv, float* __restrict__ Ls,
+                      float* __restrict__ dq_acc, int N, int n_pad, long padded_rows) {
   constexpr int kTpr = D / 8;  // threads per row
   const long gid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long row = gid / kTpr;
+  const long prow = gid / kTpr;  // row in the padded layout
   const int part = static_cast<int>(gid % kTpr);
+  const long bh = prow / n_pad;
+  const int n = static_cast<int>(prow - bh * n_pad);
+  const bool real = prow < padded_rows && n < N;
+  const long row = bh * N + n;  // row in the [B*H*N, D] tensors (when real)
   float acc = 0.f;
-  if (row < rows) {
+  if (real) {
     const uint4 o = *reinterpret_cast<const uint4*>(O + row * D + part * 8);
     const uint4 g = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
     const uint4 res = O_res != nullptr ? *reinterpret_cast<const uint4*>(O_res + row * D + part * 8)
@@ -142,9 +148,9 @@ __global__ void __launch_bounds__(256)
   }
 #pragma unroll
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (row < rows && part == 0) {
-    Dv[row] = -acc;
-    Ls[row] = L[row] * -1.4426950408889634074f;
+  if (prow < padded_rows && part == 0) {
+    Dv[prow] = real ? -acc : 0.f;
+    Ls[prow] = real ? L[row] * -1.4426950408889634074f : -INFINITY;
   }
 }
 
@@ -191,9 +197,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = N / kTile;
+  const int ntiles = (N + kTile - 1) / kTile;
   const int bh = blockIdx.x / ntiles;
   const int j = blockIdx.x - bh * ntiles;  // key tile (j = 0 has the most causal work)
+  // N % 128 != 0: rows past N arrive as zeros through the 3-D tensor maps. Padded
+  // queries have Ls = -inf, so their P is 0. Padded keys of the last key tile need no
+  // mask: their dK and dV rows are not stored, and their dS meets zero rows of K in
+  // dQ = dS K. Ls and Dv are laid out per head with ntiles * 128 rows.
   const int i_begin = CAUSAL ? j : 0;
   const int niter = ntiles - i_begin;
   const long head_row = static_cast<long>(bh) * N;
@@ -239,30 +249,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tma_prefetch(&tmV);
       tma_prefetch(&tmDO);
       tma_prefetch(&tmDQ);
-      const int krow = static_cast<int>(head_row) + j * kTile;
+
       mbar_expect_tx(bar(kBbKVFull), 2 * Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_2d(sbase + Lay::kK + c * Lay::kChunkBytes, &tmK, c * 64, krow, bar(kBbKVFull));
-        tma_load_2d(sbase + Lay::kV + c * Lay::kChunkBytes, &tmV, c * 64, krow, bar(kBbKVFull));
+        tma_load_3d(sbase + Lay::kK + c * Lay::kChunkBytes, &tmK, c * 64, j * kTile, bh,
+                    bar(kBbKVFull));
+        tma_load_3d(sbase + Lay::kV + c * Lay::kChunkBytes, &tmV, c * 64, j * kTile, bh,
+                    bar(kBbKVFull));
       }
       for (int it = 0; it < niter; ++it) {
         const int st = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
-        const int qrow = static_cast<int>(head_row) + (i_begin + it) * kTile;
+        const int qtile = (i_begin + it) * kTile;  // first query row within the head
+        const long head_pad = static_cast<long>(bh) * ntiles * kTile;  // Ls / Dv rows
         if (it >= 2 && !mbar_wait(bar(kBbQEmpty + st), (use - 1) & 1, abort_flag)) break;
         const uint32_t full = bar(kBbQFull + st);
         mbar_expect_tx(full, Lay::kTileBytes + 2 * 512);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
-                      qrow, full);
-        bulk_load(sbase + Lay::kL + st * 512, Ls + qrow, 512, full);
-        bulk_load(sbase + Lay::kDv + st * 512, Dv + qrow, 512, full);
+          tma_load_3d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
+                      qtile, bh, full);
+        bulk_load(sbase + Lay::kL + st * 512, Ls + head_pad + qtile, 512, full);
+        bulk_load(sbase + Lay::kDv + st * 512, Dv + head_pad + qtile, 512, full);
         if (it >= 1 &&
             !mbar_wait(bar(kBbDOEmpty), static_cast<uint32_t>((it - 1) & 1), abort_flag))
           break;
         mbar_expect_tx(bar(kBbDOFull), Lay::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_2d(sbase + Lay::kDO + c * Lay::kChunkBytes, &tmDO, c * 64, qrow,
+          tma_load_3d(sbase + Lay::kDO + c * Lay::kChunkBytes, &tmDO, c * 64, qtile, bh,
                       bar(kBbDOFull));
         FA_TRACE_EVENT(it, 0);
       }
@@ -476,6 +489,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       tc_fence_after();
       const long grow = head_row + static_cast<long>(j) * kTile + r;
+      const bool live_row = j * kTile + r < N;  // padded keys of the last tile are not stored
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = (which == 0 ? Lay::tDV : Lay::tDK) + half * (D / 2);
@@ -493,8 +507,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int e = 0; e < 16; ++e)
             pw[e] = pack2<BF16>(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
           uint4* dst = reinterpret_cast<uint4*>(dst_row + c * 32);
+          if (live_row) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+            for (int e = 0; e < 4; ++e) dst[e] = pk[e];
+          }
         }
       }
     }
@@ -533,7 +549,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) FA_TRACE_EVENT(it, 13);
       }
       if (!named_bar_and(5, 128, got)) break;
-      const int row = static_cast<int>(head_row) + (i_begin + it) * kTile;
+      const int qtile = (i_begin + it) * kTile;
 #pragma unroll
       for (int rnd = 0; rnd < D / 64; ++rnd) {
         if (leader) bulk_wait_read_all();  // previous round's boxes have been read
@@ -552,7 +568,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            tma_reduce_add_2d(&tmDQ, stage + h * Lay::kChunkBytes, 32 * (2 * rnd + h), row);
+            tma_reduce_add_3d(&tmDQ, stage + h * Lay::kChunkBytes, 32 * (2 * rnd + h), qtile, bh);
           bulk_commit();
         }
       }

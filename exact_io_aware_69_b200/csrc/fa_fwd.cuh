@@ -104,12 +104,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = N / kTile;
+  const int ntiles = (N + kTile - 1) / kTile;
   const int bh = blockIdx.x / ntiles;
   const int tr = blockIdx.x - bh * ntiles;
   const int t = CAUSAL ? (ntiles - 1 - tr) : tr;  // heaviest causal tiles first
   const int nkv = CAUSAL ? t + 1 : ntiles;
-  const int row0 = bh * N + t * kTile;              // first row in the [B*H*N, D] view
+  // Rows and keys of the last tile past N (when N % 128 != 0) come in as zeros from the
+  // 3-D tensor maps; the keys are masked below, the rows are not stored.
+  const int last_keys = N - (ntiles - 1) * kTile;  // valid keys in the last KV tile
 
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -151,7 +153,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch(&tmV);
       mbar_expect_tx(bar(kBarQFull), Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c)
-        tma_load_2d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, row0, bar(kBarQFull));
+        tma_load_3d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, t * kTile, bh,
+                    bar(kBarQFull));
       // step s loads K_s and V_{s-1}
       for (int step = 0; step <= nkv; ++step) {
         if (step < nkv) {
@@ -163,7 +166,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t sk = sbase + Lay::kK + ks * Lay::kTileBytes;
           mbar_expect_tx(bar(kBarKFull + ks), Lay::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sk + c * Lay::kChunkBytes, &tmK, c * 64, bh * N + step * kTile,
+            tma_load_3d(sk + c * Lay::kChunkBytes, &tmK, c * 64, step * kTile, bh,
                         bar(kBarKFull + ks));
           FA_TRACE_EVENT(step, 8);
         }
@@ -176,7 +179,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t sv = sbase + Lay::kV + vs * Lay::kTileBytes;
           mbar_expect_tx(bar(kBarVFull + vs), Lay::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_2d(sv + c * Lay::kChunkBytes, &tmV, c * 64, bh * N + j * kTile,
+            tma_load_3d(sv + c * Lay::kChunkBytes, &tmV, c * 64, j * kTile, bh,
                         bar(kBarVFull + vs));
           FA_TRACE_EVENT(j, 9);
         }
@@ -262,8 +265,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         reg_fence32(sr + 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        if (CAUSAL && j == t) {  // diagonal tile: key column > query row is masked
-          const int lim = r - half * 64;
+        // diagonal tile: key column > query row is masked; last tile: keys >= N
+        const bool diag = CAUSAL && j == t;
+        if (diag || (j == ntiles - 1 && last_keys < kTile)) {
+          int lim = (j == ntiles - 1 ? last_keys - 1 : kTile - 1) - half * 64;
+          if (diag) lim = min(lim, r - half * 64);
 #pragma unroll
           for (int c = 0; c < 64; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
         }
@@ -389,16 +395,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       fence_async_smem();
-      if (half == 0) Lse[row0 + r] = (m + log2f(l_row)) * 0.69314718055994530942f;
+      if (half == 0 && t * kTile + r < N)
+        Lse[static_cast<long>(bh) * N + t * kTile + r] =
+            (m + log2f(l_row)) * 0.69314718055994530942f;
     }
     // all 256 softmax threads have staged their part (or all gave up together)
     if (named_bar_and(5, 256, ok) && threadIdx.x == 0) {
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        tma_store_2d(&tmO, sbase + Lay::kK + c * Lay::kChunkBytes, c * 64, row0);
+        tma_store_3d(&tmO, sbase + Lay::kK + c * Lay::kChunkBytes, c * 64, t * kTile, bh);
         if (has_res)
-          tma_store_2d(&tmOres, sbase + Lay::kK + Lay::kTileBytes + c * Lay::kChunkBytes, c * 64,
-                       row0);
+          tma_store_3d(&tmOres, sbase + Lay::kK + Lay::kTileBytes + c * Lay::kChunkBytes, c * 64,
+                       t * kTile, bh);
       }
       bulk_commit();
       bulk_wait_read_all();  // shared memory is read before the CTA releases it

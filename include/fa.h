@@ -33,13 +33,15 @@
  * workspace sized by fa_bwd_workspace_size(). The library allocates no device
  * memory in these calls; its only state is one device-side error word per device.
  *
- * Supported now: d in {64, 128}; N a positive multiple of 128; dtype bf16 or fp16.
+ * Supported now: d in {64, 128}; any N >= 1 (the last 128-row tile of a head may be
+ * partial); dtype bf16 or fp16; B*H*N with N rounded up to 128 below 2^31.
  *
  * Errors are checked on the host before anything is enqueued and are returned as
  * codes (no exception, no abort, no fallback to another implementation):
  *   FA_ERR_INVALID      null pointer, negative size, misaligned pointer, a workspace
  *                       that is too small, or a non-finite / non-positive scale;
- *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, N % 128 != 0;
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, or B*H*roundup(N,128)
+ *                       >= 2^31 (32-bit TMA coordinates and grid indices);
  *   FA_ERR_CUDA         a CUDA runtime/driver call or a launch failed;
  *   FA_ERR_TIMEOUT      (from fa_get_device_status only) a kernel gave up a bounded
  *                       wait on the device and returned without finishing.
@@ -79,8 +81,9 @@ int fa_fwd(const void *Q, const void *K, const void *V, void *O, void *O_res, fl
 
 /*
  * Bytes of device workspace that fa_bwd needs for this shape: fp32 D and scaled L
- * ([B][H][N] each) plus an fp32 dQ accumulator [B][H][N][d]. 0 for an empty
- * problem; (size_t)-1 for sizes that fa_bwd rejects as invalid.
+ * ([B][H][Np] each, Np = N rounded up to a multiple of 128) plus an fp32 dQ
+ * accumulator [B][H][N][d]: B*H*Np*8 + B*H*N*d*4. 0 for an empty problem;
+ * (size_t)-1 for sizes that fa_bwd rejects as invalid.
  */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
@@ -128,10 +131,10 @@ int fa_bwd_dq_convert(void *dQ, int B, int H, int N, int d, float scale, int dty
  * 32 MiB, held on every GPU that loads the library until the process exits. It
  * calls no cudaMalloc, cudaFree or other allocating routine.
  *
- * Limit: fa_bwd_workspace_size(B, H, N, d) <= 32 MiB, i.e. B*H*N <= 64,527 at
- * d = 128 and <= 128,100 at d = 64; larger problems return FA_ERR_UNSUPPORTED
- * before anything touches the device. Other checks and results are those of
- * fa_bwd.
+ * Limit: fa_bwd_workspace_size(B, H, N, d) <= 32 MiB, i.e. (for N a multiple of 128)
+ * B*H*N <= 64,527 at d = 128 and <= 128,100 at d = 64; larger problems return
+ * FA_ERR_UNSUPPORTED before anything touches the device. Other checks and results
+ * are those of fa_bwd.
  *
  * The first call on a device looks up the scratch array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that first

@@ -94,7 +94,7 @@ def _bwd(lib, **kw):
     (dict(scale=float("inf")), fa.FA_ERR_INVALID),
     (dict(d=96), fa.FA_ERR_UNSUPPORTED),
     (dict(d=256), fa.FA_ERR_UNSUPPORTED),
-    (dict(N=200), fa.FA_ERR_UNSUPPORTED),
+    (dict(B=1 << 15, H=1 << 10, N=100), fa.FA_ERR_UNSUPPORTED),  # 2^32 padded rows
     (dict(dtype=2), fa.FA_ERR_UNSUPPORTED),
     (dict(B=0), fa.FA_OK),
     (dict(N=0, Q=None, K=None, V=None, O=None, L=None), fa.FA_OK),
@@ -112,7 +112,7 @@ def test_fwd_rejects_before_launch(lib, kw, code):
     (dict(R=P + 0xa00008), fa.FA_ERR_INVALID),
     (dict(H=-2), fa.FA_ERR_INVALID),
     (dict(d=32), fa.FA_ERR_UNSUPPORTED),
-    (dict(N=130), fa.FA_ERR_UNSUPPORTED),
+    (dict(B=1 << 20, H=16, N=130), fa.FA_ERR_UNSUPPORTED),  # 2^32 padded rows
     (dict(dtype=5), fa.FA_ERR_UNSUPPORTED),
     (dict(H=0), fa.FA_OK),
 ])
@@ -131,3 +131,14 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(fa, "_lib", None)
     with pytest.raises(ImportError):
         fa.load()
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 200, 64), (2, 3, 128, 128), (1, 1, 1, 128),
+                                     (3, 1, 8193, 64)])
+def test_workspace_size_pads_rows_per_head(lib, B, H, N, d):
+    """D and Ls take N rounded up to 128 per head; the fp32 dQ accumulator that follows
+    them starts on a 1024-byte boundary and holds exactly B*H*N*d values."""
+    n_pad = -(-N // 128) * 128
+    want = B * H * n_pad * 8 + B * H * N * d * 4
+    assert lib.fa_bwd_workspace_size(B, H, N, d) == want
+    assert (B * H * n_pad * 8) % 1024 == 0

@@ -1,6 +1,6 @@
 """CUDA path vs the fp64 oracle, element by element, at sizes the oracle finishes in
-seconds. Every shape spans several 128-row tiles; the causal cases exercise the
-diagonal-tile mask and the skipped tiles."""
+seconds. The shapes span several 128-row tiles (and, in RAGGED, end in a partial
+one); the causal cases exercise the diagonal-tile mask and the skipped tiles."""
 
 import math
 
@@ -44,6 +44,29 @@ def _run(B, H, N, d, dtype, causal, seed, large_frac=0.0):
 def test_fwd_bwd_vs_oracle(shape, causal, dtype):
     B, H, N, d = shape
     _, got, ref = _run(B, H, N, d, dtype, causal, seed=17 + N + d)
+    assert_close_L(to_f64(got["L"]), ref["L"])
+    for name in ("o", "dq", "dk", "dv"):
+        assert_close(name, to_f64(got[name]), ref[name], dtype)
+
+
+# N not a multiple of 128: the last query and key tiles are partly past the end of a
+# head (rows read as zeros, keys masked in the forward, rows not stored). 77 and 1 are
+# below one tile; 200, 333 and 1000 span several tiles and end in a ragged one.
+RAGGED = [
+    (1, 2, 200, 64),
+    (2, 1, 333, 128),
+    (1, 1, 77, 128),
+    (1, 2, 1000, 64),
+    (3, 1, 1, 128),
+]
+
+
+@pytest.mark.parametrize("dtype", [BF16, FP16])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", RAGGED, ids=lambda s: "B{}H{}N{}d{}".format(*s))
+def test_ragged_n_vs_oracle(shape, causal, dtype):
+    B, H, N, d = shape
+    _, got, ref = _run(B, H, N, d, dtype, causal, seed=91 + N + d)
     assert_close_L(to_f64(got["L"]), ref["L"])
     for name in ("o", "dq", "dk", "dv"):
         assert_close(name, to_f64(got[name]), ref[name], dtype)
