@@ -56,11 +56,16 @@ def _load():
                                     dp, dp]
     lib.oracle_attn_bwd.argtypes = [f64p, f64p, f64p, f64p, L_, L_, L_, ctypes.c_int,
                                     ctypes.c_double, dp, dp, dp, dp, dp, dp]
+    lib.oracle_attn_fwd_qk.argtypes = [f64p, f64p, f64p, L_, L_, L_, L_, ctypes.c_int,
+                                       ctypes.c_double, dp, dp]
+    lib.oracle_attn_bwd_qk.argtypes = [f64p, f64p, f64p, f64p, L_, L_, L_, L_, ctypes.c_int,
+                                       ctypes.c_double, dp, dp, dp, dp, dp, dp]
     lib.oracle_attn_rows.argtypes = [f64p, f64p, f64p, dp, L_, L_, L_, ctypes.c_int,
                                      ctypes.c_double, L_, dp, dp, dp, dp, dp, dp]
     lib.oracle_attn_keys.argtypes = [f64p, f64p, f64p, f64p, L_, L_, L_, ctypes.c_int,
                                      ctypes.c_double, L_, dp, dp, dp, dp]
-    for fn in ("oracle_attn_fwd", "oracle_attn_bwd", "oracle_attn_rows", "oracle_attn_keys"):
+    for fn in ("oracle_attn_fwd", "oracle_attn_bwd", "oracle_attn_fwd_qk", "oracle_attn_bwd_qk",
+               "oracle_attn_rows", "oracle_attn_keys"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -98,15 +103,21 @@ def _shape(q):
 
 
 def attn_fwd(q, k, v, causal: bool, scale: float):
-    """Naive attention forward. Returns (O [.., N, d] float64, L [.., N] float64)."""
+    """Naive attention forward. Returns (O [.., N_q, d] float64, L [.., N_q] float64).
+
+    k and v may have another sequence length N_k than q; causal masking is then
+    bottom-right aligned (query i sees keys j <= i + N_k - N_q), and a query row that
+    sees no key has O = 0 and L = -inf.
+    """
     lib = _load()
     shp = q.shape
-    BH, N, d = _shape(q)
+    BH, Nq, d = _shape(q)
+    Nk = _shape(k)[1]
     q, k, v = _f64(q), _f64(k), _f64(v)
-    o = np.empty((BH, N, d), np.float64)
-    L = np.empty((BH, N), np.float64)
-    _check(lib.oracle_attn_fwd(q, k, v, BH, N, d, int(causal), float(scale), _ptr(o), _ptr(L)),
-           "oracle_attn_fwd")
+    o = np.empty((BH, Nq, d), np.float64)
+    L = np.empty((BH, Nq), np.float64)
+    _check(lib.oracle_attn_fwd_qk(q, k, v, BH, Nq, Nk, d, int(causal), float(scale), _ptr(o),
+                                  _ptr(L)), "oracle_attn_fwd_qk")
     return o.reshape(shp), L.reshape(shp[:-1])
 
 
@@ -114,19 +125,26 @@ def attn_bwd(q, k, v, do, causal: bool, scale: float):
     """Naive attention forward and analytic backward.
 
     Returns a dict with float64 arrays o, L, dq, dk, dv and D (= sum_j P_ij dP_ij).
+    k and v may be longer or shorter than q, as in attn_fwd; dk and dv then have k's
+    shape.
     """
     lib = _load()
-    shp = q.shape
-    BH, N, d = _shape(q)
+    shp, kshp = q.shape, k.shape
+    BH, Nq, d = _shape(q)
+    Nk = _shape(k)[1]
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
-    out = {name: np.empty((BH, N, d), np.float64) for name in ("o", "dq", "dk", "dv")}
-    out["L"] = np.empty((BH, N), np.float64)
-    out["D"] = np.empty((BH, N), np.float64)
-    _check(lib.oracle_attn_bwd(q, k, v, do, BH, N, d, int(causal), float(scale),
-                               _ptr(out["o"]), _ptr(out["L"]), _ptr(out["dq"]), _ptr(out["dk"]),
-                               _ptr(out["dv"]), _ptr(out["D"])), "oracle_attn_bwd")
-    for name in ("o", "dq", "dk", "dv"):
+    out = {name: np.empty((BH, Nq, d), np.float64) for name in ("o", "dq")}
+    out.update({name: np.empty((BH, Nk, d), np.float64) for name in ("dk", "dv")})
+    out["L"] = np.empty((BH, Nq), np.float64)
+    out["D"] = np.empty((BH, Nq), np.float64)
+    _check(lib.oracle_attn_bwd_qk(q, k, v, do, BH, Nq, Nk, d, int(causal), float(scale),
+                                  _ptr(out["o"]), _ptr(out["L"]), _ptr(out["dq"]),
+                                  _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["D"])),
+           "oracle_attn_bwd_qk")
+    for name in ("o", "dq"):
         out[name] = out[name].reshape(shp)
+    for name in ("dk", "dv"):
+        out[name] = out[name].reshape(kshp)
     out["L"] = out["L"].reshape(shp[:-1])
     out["D"] = out["D"].reshape(shp[:-1])
     return out

@@ -26,8 +26,11 @@
  *                                         recordar": only per-row statistics survive)
  *
  * Causal masking (a reading, not on the pages): key j is visible to query i iff
- * j <= i, with N_q = N_k = N; masked scores do not enter the max or the sum, so
- * P_ij = 0 there. Row i always sees key i, so no row is empty.
+ * j <= i + (N_k - N_q), i.e. the last query sees every key ("bottom-right"
+ * alignment; with N_q = N_k this is j <= i). Masked scores do not enter the max or
+ * the sum, so P_ij = 0 there. With N_q > N_k the first N_q - N_k queries see no key
+ * at all; their rows are defined as O_i = 0, L_i = -inf, dQ_i = 0, D_i = 0 (the
+ * empty sum), and they add nothing to dK or dV.
  *
  * Backward, given dO (standard calculus of the three steps above; the pages say only
  * that the gradient needs P and that P is recomputed from Q, K, V):
@@ -39,7 +42,8 @@
  *   dQ_i  = scale * sum_j dS_ij k_j
  *   dK_j  = scale * sum_i dS_ij q_i
  *
- * Inputs are double arrays [BH][N][d]; for parity checks they hold the exact 16-bit
+ * Inputs are double arrays, q and dO [BH][N_q][d], k and v [BH][N_k][d] (the
+ * square entry points take N_q = N_k = N); for parity checks they hold the exact 16-bit
  * values used on the GPU (widening is exact). Every product and sum is taken in
  * double, and outputs are double.
  *
@@ -73,8 +77,12 @@ void oracle_set_threads(int n) {
 #endif
 }
 
-/* Number of keys that query row i sees. */
-static long visible_keys(long i, long N, int causal) { return causal ? i + 1 : N; }
+/* Number of keys that query row i sees: a prefix of the Nk keys. */
+static long visible_keys(long i, long Nq, long Nk, int causal) {
+    if (!causal) return Nk;
+    const long n = i + 1 + (Nk - Nq);
+    return n < 0 ? 0 : (n > Nk ? Nk : n);
+}
 
 /* s[j] = scale * (q_i . k_j) for the first nvis keys of one head. */
 static void score_row(const double *qi, const double *kh, long nvis, long d, double scale,
@@ -97,8 +105,9 @@ static void softmax_row(double *s, long nvis, double *m_out, double *l_out) {
         s[j] = exp(s[j] - m);
         l += s[j];
     }
-    for (long j = 0; j < nvis; ++j) s[j] /= l;
-    *m_out = m;
+    if (nvis > 0)
+        for (long j = 0; j < nvis; ++j) s[j] /= l;
+    *m_out = m;  /* -inf and 0 for a row that sees no key */
     *l_out = l;
 }
 
@@ -117,9 +126,10 @@ static void weighted_rows(const double *w, const double *xh, long nvis, long d, 
  * and, when doi != NULL, dP_i (left in dp), D_i and dQ_i.
  */
 static void query_row(const double *qh, const double *kh, const double *vh, const double *doh,
-                      long N, long d, int causal, double scale, long i, double *p, double *dp,
-                      double *o_i, double *m_i, double *l_i, double *D_i, double *dq_i) {
-    const long nvis = visible_keys(i, N, causal);
+                      long Nq, long Nk, long d, int causal, double scale, long i, double *p,
+                      double *dp, double *o_i, double *m_i, double *l_i, double *D_i,
+                      double *dq_i) {
+    const long nvis = visible_keys(i, Nq, Nk, causal);
     const double *qi = qh + i * d;
     score_row(qi, kh, nvis, d, scale, p);
     softmax_row(p, nvis, m_i, l_i);
@@ -143,37 +153,43 @@ static void query_row(const double *qh, const double *kh, const double *vh, cons
     }
 }
 
-static int check_args(const void *q, const void *k, const void *v, long BH, long N, long d) {
+static int check_args(const void *q, const void *k, const void *v, long BH, long Nq, long Nk,
+                      long d) {
     if (!q || !k || !v) return ORC_EINVAL;
-    if (BH < 0 || N < 0 || d <= 0) return ORC_EINVAL;
+    if (BH < 0 || Nq < 0 || Nk < 0 || d <= 0) return ORC_EINVAL;
     return ORC_OK;
 }
 
-/* Forward: o [BH][N][d] and L [BH][N] (either may be NULL). */
-int oracle_attn_fwd(const double *q, const double *k, const double *v, long BH, long N, long d,
-                    int causal, double scale, double *o, double *L) {
-    if (check_args(q, k, v, BH, N, d)) return ORC_EINVAL;
+/* Forward: o [BH][Nq][d] and L [BH][Nq] (either may be NULL). */
+int oracle_attn_fwd_qk(const double *q, const double *k, const double *v, long BH, long Nq,
+                       long Nk, long d, int causal, double scale, double *o, double *L) {
+    if (check_args(q, k, v, BH, Nq, Nk, d)) return ORC_EINVAL;
     int err = ORC_OK;
 #pragma omp parallel
     {
-        double *p = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
         if (!p) {
 #pragma omp atomic write
             err = ORC_ENOMEM;
         }
 #pragma omp for schedule(dynamic, 16) collapse(2)
         for (long bh = 0; bh < BH; ++bh)
-            for (long i = 0; i < N; ++i) {
+            for (long i = 0; i < Nq; ++i) {
                 if (!p) continue;
-                const size_t h = (size_t)bh * N * d;
+                const size_t hq = (size_t)bh * Nq * d, hk = (size_t)bh * Nk * d;
                 double m, l;
-                query_row(q + h, k + h, v + h, NULL, N, d, causal, scale, i, p, NULL,
-                          o ? o + h + (size_t)i * d : NULL, &m, &l, NULL, NULL);
-                if (L) L[(size_t)bh * N + i] = m + log(l);
+                query_row(q + hq, k + hk, v + hk, NULL, Nq, Nk, d, causal, scale, i, p, NULL,
+                          o ? o + hq + (size_t)i * d : NULL, &m, &l, NULL, NULL);
+                if (L) L[(size_t)bh * Nq + i] = m + log(l);
             }
         free(p);
     }
     return err;
+}
+
+int oracle_attn_fwd(const double *q, const double *k, const double *v, long BH, long N, long d,
+                    int causal, double scale, double *o, double *L) {
+    return oracle_attn_fwd_qk(q, k, v, BH, N, N, d, causal, scale, o, L);
 }
 
 /*
@@ -196,8 +212,8 @@ static int head_row_stats(const double *qh, const double *kh, const double *vh, 
 #pragma omp for schedule(dynamic, 16)
         for (long i = i0; i < N; ++i) {
             if (!p || !dp) continue;
-            query_row(qh, kh, vh, doh, N, d, causal, scale, i, p, dp, NULL, &m[i], &l[i], &D[i],
-                      NULL);
+            query_row(qh, kh, vh, doh, N, N, d, causal, scale, i, p, dp, NULL, &m[i], &l[i],
+                      &D[i], NULL);
         }
         free(p);
         free(dp);
@@ -210,12 +226,15 @@ static int head_row_stats(const double *qh, const double *kh, const double *vh, 
  * P_ij = exp(s_ij - m_i) / l_i for every row i that sees key j.
  */
 static void key_grads(const double *qh, const double *kh, const double *vh, const double *doh,
-                      long N, long d, int causal, double scale, long j, const double *m,
+                      long Nq, long Nk, long d, int causal, double scale, long j, const double *m,
                       const double *l, const double *D, double *dk_j, double *dv_j) {
     const double *kj = kh + j * d;
     const double *vj = vh + j * d;
     for (long t = 0; t < d; ++t) dk_j[t] = dv_j[t] = 0.0;
-    for (long i = causal ? j : 0; i < N; ++i) {
+    /* rows that see key j: i + (Nk - Nq) >= j */
+    long i0 = causal ? j - (Nk - Nq) : 0;
+    if (i0 < 0) i0 = 0;
+    for (long i = i0; i < Nq; ++i) {
         const double *qi = qh + i * d;
         const double *doi = doh + i * d;
         double s = 0.0, dp = 0.0;
@@ -237,44 +256,44 @@ static void key_grads(const double *qh, const double *kh, const double *vh, cons
  * Forward and backward for every head. o, L, dq, dk, dv, D may each be NULL.
  * Row-wise quantities first, then key-wise ones (dK, dV) from the stored m, l, D.
  */
-int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO, long BH,
-                    long N, long d, int causal, double scale, double *o, double *L, double *dq,
-                    double *dk, double *dv, double *D_out) {
-    if (check_args(q, k, v, BH, N, d) || !dO) return ORC_EINVAL;
-    if (N == 0 || BH == 0) return ORC_OK;
-    double *m = (double *)malloc(sizeof(double) * (size_t)N);
-    double *l = (double *)malloc(sizeof(double) * (size_t)N);
-    double *D = (double *)malloc(sizeof(double) * (size_t)N);
+int oracle_attn_bwd_qk(const double *q, const double *k, const double *v, const double *dO,
+                       long BH, long Nq, long Nk, long d, int causal, double scale, double *o,
+                       double *L, double *dq, double *dk, double *dv, double *D_out) {
+    if (check_args(q, k, v, BH, Nq, Nk, d) || !dO) return ORC_EINVAL;
+    if (Nq == 0 || Nk == 0 || BH == 0) return ORC_OK;
+    double *m = (double *)malloc(sizeof(double) * (size_t)Nq);
+    double *l = (double *)malloc(sizeof(double) * (size_t)Nq);
+    double *D = (double *)malloc(sizeof(double) * (size_t)Nq);
     if (!m || !l || !D) {
         free(m); free(l); free(D);
         return ORC_ENOMEM;
     }
     int err = ORC_OK;
     for (long bh = 0; bh < BH && err == ORC_OK; ++bh) {
-        const size_t h = (size_t)bh * N * d;
-        const double *qh = q + h, *kh = k + h, *vh = v + h, *doh = dO + h;
+        const size_t hq = (size_t)bh * Nq * d, hk = (size_t)bh * Nk * d;
+        const double *qh = q + hq, *kh = k + hk, *vh = v + hk, *doh = dO + hq;
 #pragma omp parallel
         {
-            double *p = (double *)malloc(sizeof(double) * (size_t)N);
-            double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+            double *p = (double *)malloc(sizeof(double) * (size_t)Nk);
+            double *dp = (double *)malloc(sizeof(double) * (size_t)Nk);
             if (!p || !dp) {
 #pragma omp atomic write
                 err = ORC_ENOMEM;
             }
 #pragma omp for schedule(dynamic, 8)
-            for (long i = 0; i < N; ++i) {
+            for (long i = 0; i < Nq; ++i) {
                 if (!p || !dp) continue;
-                query_row(qh, kh, vh, doh, N, d, causal, scale, i, p, dp,
-                          o ? o + h + (size_t)i * d : NULL, &m[i], &l[i], &D[i],
-                          dq ? dq + h + (size_t)i * d : NULL);
+                query_row(qh, kh, vh, doh, Nq, Nk, d, causal, scale, i, p, dp,
+                          o ? o + hq + (size_t)i * d : NULL, &m[i], &l[i], &D[i],
+                          dq ? dq + hq + (size_t)i * d : NULL);
             }
             free(p);
             free(dp);
         }
         if (err != ORC_OK) break;
-        for (long i = 0; i < N; ++i) {
-            if (L) L[(size_t)bh * N + i] = m[i] + log(l[i]);
-            if (D_out) D_out[(size_t)bh * N + i] = D[i];
+        for (long i = 0; i < Nq; ++i) {
+            if (L) L[(size_t)bh * Nq + i] = m[i] + log(l[i]);
+            if (D_out) D_out[(size_t)bh * Nq + i] = D[i];
         }
         if (dk || dv) {
 #pragma omp parallel
@@ -286,11 +305,11 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
                     err = ORC_ENOMEM;
                 }
 #pragma omp for schedule(dynamic, 8)
-                for (long j = 0; j < N; ++j) {
+                for (long j = 0; j < Nk; ++j) {
                     if (!gk || !gv) continue;
-                    key_grads(qh, kh, vh, doh, N, d, causal, scale, j, m, l, D, gk, gv);
-                    if (dk) memcpy(dk + h + (size_t)j * d, gk, sizeof(double) * (size_t)d);
-                    if (dv) memcpy(dv + h + (size_t)j * d, gv, sizeof(double) * (size_t)d);
+                    key_grads(qh, kh, vh, doh, Nq, Nk, d, causal, scale, j, m, l, D, gk, gv);
+                    if (dk) memcpy(dk + hk + (size_t)j * d, gk, sizeof(double) * (size_t)d);
+                    if (dv) memcpy(dv + hk + (size_t)j * d, gv, sizeof(double) * (size_t)d);
                 }
                 free(gk);
                 free(gv);
@@ -301,6 +320,12 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
     return err;
 }
 
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dO, long BH,
+                    long N, long d, int causal, double scale, double *o, double *L, double *dq,
+                    double *dk, double *dv, double *D_out) {
+    return oracle_attn_bwd_qk(q, k, v, dO, BH, N, N, d, causal, scale, o, L, dq, dk, dv, D_out);
+}
+
 /*
  * Selected query rows only, each in O(N d): for n pairs (bh_sel[r], row_sel[r])
  * write o[r][d], L[r], and when dO != NULL also dq[r][d] and D[r].
@@ -308,7 +333,7 @@ int oracle_attn_bwd(const double *q, const double *k, const double *v, const dou
 int oracle_attn_rows(const double *q, const double *k, const double *v, const double *dO, long BH,
                      long N, long d, int causal, double scale, long n, const long *bh_sel,
                      const long *row_sel, double *o, double *L, double *dq, double *D) {
-    if (check_args(q, k, v, BH, N, d) || n < 0 || (n > 0 && (!bh_sel || !row_sel)))
+    if (check_args(q, k, v, BH, N, N, d) || n < 0 || (n > 0 && (!bh_sel || !row_sel)))
         return ORC_EINVAL;
     for (long r = 0; r < n; ++r)
         if (bh_sel[r] < 0 || bh_sel[r] >= BH || row_sel[r] < 0 || row_sel[r] >= N)
@@ -327,8 +352,8 @@ int oracle_attn_rows(const double *q, const double *k, const double *v, const do
             if (!p || !dp) continue;
             const size_t h = (size_t)bh_sel[r] * N * d;
             double m, l, Dr = 0.0;
-            query_row(q + h, k + h, v + h, dO ? dO + h : NULL, N, d, causal, scale, row_sel[r], p,
-                      dp, o ? o + (size_t)r * d : NULL, &m, &l, &Dr,
+            query_row(q + h, k + h, v + h, dO ? dO + h : NULL, N, N, d, causal, scale, row_sel[r],
+                      p, dp, o ? o + (size_t)r * d : NULL, &m, &l, &Dr,
                       (dO && dq) ? dq + (size_t)r * d : NULL);
             if (L) L[r] = m + log(l);
             if (D) D[r] = Dr;
@@ -348,7 +373,7 @@ int oracle_attn_rows(const double *q, const double *k, const double *v, const do
 int oracle_attn_keys(const double *q, const double *k, const double *v, const double *dO, long BH,
                      long N, long d, int causal, double scale, long n, const long *bh_sel,
                      const long *key_sel, double *dk, double *dv) {
-    if (check_args(q, k, v, BH, N, d) || !dO || n < 0 || (n > 0 && (!bh_sel || !key_sel)))
+    if (check_args(q, k, v, BH, N, N, d) || !dO || n < 0 || (n > 0 && (!bh_sel || !key_sel)))
         return ORC_EINVAL;
     for (long r = 0; r < n; ++r)
         if (bh_sel[r] < 0 || bh_sel[r] >= BH || key_sel[r] < 0 || key_sel[r] >= N)
@@ -375,7 +400,7 @@ int oracle_attn_keys(const double *q, const double *k, const double *v, const do
 #pragma omp parallel for schedule(dynamic, 1)
         for (long r = r0; r < n; ++r) {
             if (bh_sel[r] != bh) continue;
-            key_grads(q + h, k + h, v + h, dO + h, N, d, causal, scale, key_sel[r], m, l, D,
+            key_grads(q + h, k + h, v + h, dO + h, N, N, d, causal, scale, key_sel[r], m, l, D,
                       dk + (size_t)r * d, dv + (size_t)r * d);
             done[r] = 1;
         }

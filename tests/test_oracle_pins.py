@@ -297,3 +297,77 @@ def test_scale_enters_scores():
     o2, L2 = oracle.attn_fwd(q, k, v, False, 2.0)
     np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(L1, L2, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- N_q != N_k
+# Bottom-right causal alignment (query i sees keys j <= i + N_k - N_q) and rows that
+# see no key, pinned to independent results: SciPy's softmax for a single query, and
+# the square causal oracle (pinned above) through the identities below.
+
+def _qkv(nq, nk, d, seed, bh=2):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((bh, nq, d))
+    k = rng.standard_normal((bh, nk, d))
+    v = rng.standard_normal((bh, nk, d))
+    do = rng.standard_normal((bh, nq, d))
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_query_is_library_softmax(causal):
+    """N_q = 1: the query sees every key either way; O = softmax(scale K q) V and
+    L = logsumexp(scale K q) by SciPy."""
+    from scipy.special import logsumexp, softmax
+    q, k, v, _ = _qkv(1, 37, 16, seed=5)
+    scale = 0.3
+    o, L = oracle.attn_fwd(q, k, v, causal, scale)
+    for h in range(q.shape[0]):
+        s = scale * k[h] @ q[h, 0]
+        np.testing.assert_allclose(o[h, 0], softmax(s) @ v[h], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(L[h, 0], logsumexp(s), rtol=1e-13)
+
+
+def test_non_causal_rows_are_independent():
+    """Without a mask each query row is its own single-query problem."""
+    q, k, v, _ = _qkv(5, 23, 8, seed=6)
+    o, L = oracle.attn_fwd(q, k, v, False, 0.4)
+    for i in range(q.shape[1]):
+        oi, Li = oracle.attn_fwd(q[:, i:i + 1], k, v, False, 0.4)
+        np.testing.assert_array_equal(o[:, i:i + 1], oi)
+        np.testing.assert_array_equal(L[:, i:i + 1], Li)
+
+
+@pytest.mark.parametrize("nq,nk", [(3, 11), (7, 8), (1, 5)])
+def test_bottom_right_causal_is_suffix_of_square(nq, nk):
+    """N_q < N_k, causal: the rows equal the last N_q rows of the square causal problem
+    whose queries are [any N_k - N_q rows; Q]; with dO = [0; dO] the extra rows add
+    nothing to dK and dV either."""
+    q, k, v, do = _qkv(nq, nk, 8, seed=nq * 31 + nk)
+    rng = np.random.default_rng(99)
+    extra = rng.standard_normal((q.shape[0], nk - nq, q.shape[2]))
+    q_sq = np.concatenate([extra, q], axis=1)
+    do_sq = np.concatenate([np.zeros_like(extra), do], axis=1)
+    got = oracle.attn_bwd(q, k, v, do, True, 0.35)
+    sq = oracle.attn_bwd(q_sq, k, v, do_sq, True, 0.35)
+    for name in ("o", "dq"):
+        np.testing.assert_allclose(got[name], sq[name][:, nk - nq:], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(got["L"], sq["L"][:, nk - nq:], rtol=1e-13)
+    for name in ("dk", "dv"):
+        np.testing.assert_allclose(got[name], sq[name], rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,nk", [(9, 4), (6, 1)])
+def test_queries_that_see_no_key(nq, nk):
+    """N_q > N_k, causal: the first N_q - N_k queries see no key (O = 0, L = -inf,
+    dQ = 0, D = 0, nothing added to dK, dV); the others are the square causal problem
+    on the last N_k queries."""
+    q, k, v, do = _qkv(nq, nk, 8, seed=nq * 7 + nk)
+    got = oracle.attn_bwd(q, k, v, do, True, 0.5)
+    e = nq - nk
+    assert np.all(got["o"][:, :e] == 0) and np.all(got["dq"][:, :e] == 0)
+    assert np.all(got["L"][:, :e] == -np.inf) and np.all(got["D"][:, :e] == 0)
+    sq = oracle.attn_bwd(q[:, e:], k, v, do[:, e:], True, 0.5)
+    for name in ("o", "dq", "L", "D"):
+        np.testing.assert_array_equal(got[name][:, e:], sq[name])
+    for name in ("dk", "dv"):
+        np.testing.assert_allclose(got[name], sq[name], rtol=1e-13, atol=1e-15)
