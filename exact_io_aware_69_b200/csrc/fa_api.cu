@@ -82,28 +82,36 @@ bool make_tmap_f32(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Shape checks shared by fa_fwd and fa_bwd. Returns FA_OK to proceed, or an error;
-// *empty is set for a valid problem with no work.
-int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty) {
+// Shape checks shared by the forward and backward entry points. Returns FA_OK to
+// proceed, or an error; *empty is set for a valid problem with no query rows (the
+// backward then still owes dK = dV = 0 when Nk > 0). Keys are required when there are
+// queries: a row with no key at all has no softmax.
+int check_shape_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale, bool* empty) {
   *empty = false;
-  if (B < 0 || H < 0 || N < 0 || d < 0) return FA_ERR_INVALID;
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return FA_ERR_INVALID;
   if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H * N == 0) {
+  if (static_cast<long long>(B) * H * Nq == 0) {
     *empty = true;
     return FA_OK;
   }
+  if (Nk == 0) return FA_ERR_INVALID;
   // TMA coordinates and grid indices are 32-bit (rows counted with N padded to 128)
-  if (static_cast<long long>(B) * H * ((N + fa::kTile - 1) / fa::kTile * fa::kTile) >= (1LL << 31))
+  const long long pq = (Nq + fa::kTile - 1) / fa::kTile * fa::kTile;
+  const long long pk = (Nk + fa::kTile - 1) / fa::kTile * fa::kTile;
+  if (static_cast<long long>(B) * H * (pq > pk ? pq : pk) >= (1LL << 31))
     return FA_ERR_UNSUPPORTED;
   return FA_OK;
+}
+int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty) {
+  return check_shape_qk(B, H, N, N, d, dtype, scale, empty);
 }
 
 template <int D, bool CAUSAL, bool BF16>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int BH,
-               int N, float scale, cudaStream_t stream) {
+               int Nq, int Nk, float scale, cudaStream_t stream) {
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, BF16>;
   // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
   // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
@@ -112,8 +120,8 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
       cudaSuccess)
     return FA_ERR_CUDA;
   const unsigned grid =
-      static_cast<unsigned>(BH) * static_cast<unsigned>((N + fa::kTile - 1) / fa::kTile);
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, N,
+      static_cast<unsigned>(BH) * static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk,
                                                  scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -132,7 +140,8 @@ struct BwdArgs {
   void* dK;
   void* dV;
   int BH;
-  int N;
+  int Nq;  // query rows (Q, O, dO, dQ, L, the workspace)
+  int Nk;  // key rows (K, V, dK, dV)
   float scale;
   void* workspace;
   cudaStream_t stream;
@@ -140,12 +149,12 @@ struct BwdArgs {
 
 enum { kStagePre = 1, kStageMain = 2, kStageDq = 4, kStageAll = 7 };
 
-// Workspace: D and Ls as [BH][n_pad] fp32 (n_pad = N rounded up to 128, so that every
-// query tile reads whole 512-byte rows), then the dQ accumulator [BH][N][d] fp32.
+// Workspace: D and Ls as [BH][n_pad] fp32 (n_pad = Nq rounded up to 128, so that every
+// query tile reads whole 512-byte rows), then the dQ accumulator [BH][Nq][d] fp32.
 template <int D, bool CAUSAL, bool BF16>
 int launch_bwd(const BwdArgs& a, int stages) {
-  const long rows = static_cast<long>(a.BH) * a.N;
-  const int n_pad = (a.N + fa::kTile - 1) / fa::kTile * fa::kTile;
+  const long rows = static_cast<long>(a.BH) * a.Nq;
+  const int n_pad = (a.Nq + fa::kTile - 1) / fa::kTile * fa::kTile;
   const long prows = static_cast<long>(a.BH) * n_pad;
   float* Dv = static_cast<float*>(a.workspace);
   float* Ls = Dv + prows;
@@ -155,7 +164,7 @@ int launch_bwd(const BwdArgs& a, int stages) {
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
         static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.O_res),
-        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, a.N, n_pad, prows);
+        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, a.Nq, n_pad, prows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stages & kStageMain) {
@@ -172,10 +181,11 @@ int launch_bwd(const BwdArgs& a, int stages) {
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FA_ERR_CUDA;
     if (attr.numRegs != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
-    const unsigned grid = static_cast<unsigned>(prows / fa::kTile);
+    const unsigned grid =  // one CTA per key tile
+        static_cast<unsigned>(a.BH) * static_cast<unsigned>((a.Nk + fa::kTile - 1) / fa::kTile);
     kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
         *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
-        static_cast<uint16_t*>(a.dV), a.N, a.scale, a.scale * 1.4426950408889634074f,
+        static_cast<uint16_t*>(a.dV), a.Nq, a.Nk, a.scale, a.scale * 1.4426950408889634074f,
         static_cast<uint32_t>(smem));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
@@ -261,10 +271,11 @@ const char* fa_status_string(int status) {
   }
 }
 
-int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L, int B,
-           int H, int N, int d, int causal, float scale, int dtype, void* stream) {
+int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L,
+              int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
+              void* stream) {
   bool empty;
-  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  int st = check_shape_qk(B, H, Nq, Nk, d, dtype, scale, &empty);
   if (st != FA_OK || empty) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L) ||
@@ -272,12 +283,17 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, fl
     return FA_ERR_INVALID;
   const int BH = B * H;
   CUtensorMap tq, tk, tv, to, tr;
-  if (!make_tmap(&tq, Q, BH, N, d, dtype) || !make_tmap(&tk, K, BH, N, d, dtype) ||
-      !make_tmap(&tv, V, BH, N, d, dtype) || !make_tmap(&to, O, BH, N, d, dtype) ||
-      !make_tmap(&tr, O_res != nullptr ? O_res : O, BH, N, d, dtype))
+  if (!make_tmap(&tq, Q, BH, Nq, d, dtype) || !make_tmap(&tk, K, BH, Nk, d, dtype) ||
+      !make_tmap(&tv, V, BH, Nk, d, dtype) || !make_tmap(&to, O, BH, Nq, d, dtype) ||
+      !make_tmap(&tr, O_res != nullptr ? O_res : O, BH, Nq, d, dtype))
     return FA_ERR_CUDA;
-  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, B * H, N,
+  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, BH, Nq, Nk,
                           scale, static_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L, int B,
+           int H, int N, int d, int causal, float scale, int dtype, void* stream) {
+  return fa_fwd_qk(Q, K, V, O, O_res, L, B, H, N, N, d, causal, scale, dtype, stream);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -293,47 +309,71 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 
 // Validation shared by fa_bwd and its stages; the pointers a stage does not use may
 // be NULL (checked by the caller).
-static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* workspace,
-               size_t workspace_bytes, bool* empty) {
-  int st = check_shape(B, H, N, d, dtype, scale, empty);
+static int bwd_common_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale,
+                         void* workspace, size_t workspace_bytes, bool* empty) {
+  int st = check_shape_qk(B, H, Nq, Nk, d, dtype, scale, empty);
   if (st != FA_OK || *empty) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID;
-  if (workspace_bytes < fa_bwd_workspace_size(B, H, N, d)) return FA_ERR_INVALID;
+  if (workspace_bytes < fa_bwd_workspace_size(B, H, Nq, d)) return FA_ERR_INVALID;
   return FA_OK;
 }
+static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* workspace,
+                      size_t workspace_bytes, bool* empty) {
+  return bwd_common_qk(B, H, N, N, d, dtype, scale, workspace, workspace_bytes, empty);
+}
 
-static int bwd_run(const void* Q, const void* K, const void* V, const void* O,
-            const void* O_res, const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
-            int causal, float scale, int dtype, void* workspace, void* stream, int stages) {
+static int bwd_run(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
+                   const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H,
+                   int Nq, int Nk, int d, int causal, float scale, int dtype, void* workspace,
+                   void* stream, int stages) {
   const int BH = B * H;
-  const long prows = static_cast<long>(BH) * ((N + fa::kTile - 1) / fa::kTile * fa::kTile);
+  const long prows = static_cast<long>(BH) * ((Nq + fa::kTile - 1) / fa::kTile * fa::kTile);
   CUtensorMap tq, tk, tv, tdo, tdq;
   if (stages & kStageMain) {
     const float* dq_acc = static_cast<const float*>(workspace) + 2 * prows;
-    if (!make_tmap(&tq, Q, BH, N, d, dtype) || !make_tmap(&tk, K, BH, N, d, dtype) ||
-        !make_tmap(&tv, V, BH, N, d, dtype) || !make_tmap(&tdo, dO, BH, N, d, dtype) ||
-        !make_tmap_f32(&tdq, dq_acc, BH, N, d))
+    if (!make_tmap(&tq, Q, BH, Nq, d, dtype) || !make_tmap(&tk, K, BH, Nk, d, dtype) ||
+        !make_tmap(&tv, V, BH, Nk, d, dtype) || !make_tmap(&tdo, dO, BH, Nq, d, dtype) ||
+        !make_tmap_f32(&tdq, dq_acc, BH, Nq, d))
       return FA_ERR_CUDA;
   }
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, O, O_res, dO, L, dQ, dK, dV, B * H, N, scale, workspace,
+  BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, O, O_res, dO, L, dQ, dK, dV, BH, Nq, Nk, scale, workspace,
             static_cast<cudaStream_t>(stream)};
   return dispatch<BwdRun>(d, causal, dtype, a, stages);
 }
 
 static bool ok_ptr(const void* p) { return p && aligned16(p); }
 
+int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
+              const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq,
+              int Nk, int d, int causal, float scale, int dtype, void* workspace,
+              size_t workspace_bytes, void* stream) {
+  bool empty;
+  int st = bwd_common_qk(B, H, Nq, Nk, d, dtype, scale, workspace, workspace_bytes, &empty);
+  if (st != FA_OK) return st;
+  if (empty) {
+    // no query rows: every key's gradient is an empty sum
+    const size_t bytes = static_cast<size_t>(B) * H * Nk * d * 2;
+    if (bytes == 0) return FA_OK;
+    if (!ok_ptr(dK) || !ok_ptr(dV)) return FA_ERR_INVALID;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return cudaMemsetAsync(dK, 0, bytes, s) == cudaSuccess &&
+                   cudaMemsetAsync(dV, 0, bytes, s) == cudaSuccess
+               ? FA_OK
+               : FA_ERR_CUDA;
+  }
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
+      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
+    return FA_ERR_INVALID;
+  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, Nq, Nk, d, causal, scale, dtype,
+                 workspace, stream, kStageAll);
+}
+
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
            const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int N,
            int d, int causal, float scale, int dtype, void* workspace, size_t workspace_bytes,
            void* stream) {
-  bool empty;
-  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
-  if (st != FA_OK || empty) return st;
-  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
-      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
-    return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype,
-                 workspace, stream, kStageAll);
+  return fa_bwd_qk(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, N, d, causal, scale, dtype,
+                   workspace, workspace_bytes, stream);
 }
 
 int fa_bwd_preprocess(const void* O, const void* O_res, const void* dO, const float* L, int B,
@@ -344,7 +384,7 @@ int fa_bwd_preprocess(const void* O, const void* O_res, const void* dO, const fl
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) || !aligned16(O_res)) return FA_ERR_INVALID;
   return bwd_run(nullptr, nullptr, nullptr, O, O_res, dO, L, nullptr, nullptr, nullptr, B, H, N,
-                 d, 0, 1.f, dtype, workspace, stream, kStagePre);
+                 N, d, 0, 1.f, dtype, workspace, stream, kStagePre);
 }
 
 int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
@@ -355,7 +395,7 @@ int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, voi
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO) || !ok_ptr(dK) || !ok_ptr(dV))
     return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, nullptr, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, d, causal,
+  return bwd_run(Q, K, V, nullptr, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, N, d, causal,
                  scale, dtype, workspace, stream, kStageMain);
 }
 
@@ -366,7 +406,7 @@ int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dty
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(dQ)) return FA_ERR_INVALID;
   return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
-                 nullptr, B, H, N, d, 0, scale, dtype, workspace, stream, kStageDq);
+                 nullptr, B, H, N, N, d, 0, scale, dtype, workspace, stream, kStageDq);
 }
 
 int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
@@ -386,7 +426,7 @@ int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
     return FA_ERR_INVALID;
   void* scratch = noalloc_scratch_address(&st);
   if (st != FA_OK) return st;
-  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype,
+  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, N, d, causal, scale, dtype,
                  scratch, stream, kStageAll);
 }
 

@@ -150,7 +150,8 @@ __global__ void __launch_bounds__(256)
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (prow < padded_rows && part == 0) {
     Dv[prow] = real ? -acc : 0.f;
-    Ls[prow] = real ? L[row] * -1.4426950408889634074f : -INFINITY;
+    // -L log2(e); a row that sees no key (L = -inf) gets -inf too, so that its p is 0
+    Ls[prow] = (real && L[row] != -INFINITY) ? L[row] * -1.4426950408889634074f : -INFINITY;
   }
 }
 
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tmDO,
                        const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ Ls,
                        const float* __restrict__ Dv, float* __restrict__ dq_acc,
-                       uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int N,
+                       uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int Nq, int Nk,
                        float scale, float scale_log2, uint32_t smem_alloc) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -197,16 +198,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = (N + kTile - 1) / kTile;
-  const int bh = blockIdx.x / ntiles;
-  const int j = blockIdx.x - bh * ntiles;  // key tile (j = 0 has the most causal work)
-  // N % 128 != 0: rows past N arrive as zeros through the 3-D tensor maps. Padded
-  // queries have Ls = -inf, so their P is 0. Padded keys of the last key tile need no
-  // mask: their dK and dV rows are not stored, and their dS meets zero rows of K in
-  // dQ = dS K. Ls and Dv are laid out per head with ntiles * 128 rows.
-  const int i_begin = CAUSAL ? j : 0;
-  const int niter = ntiles - i_begin;
-  const long head_row = static_cast<long>(bh) * N;
+  const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head
+  const int ntk = (Nk + kTile - 1) / kTile;  // key tiles per head (one CTA each)
+  const int bh = blockIdx.x / ntk;
+  const int j = blockIdx.x - bh * ntk;  // key tile (j = 0 has the most causal work)
+  // Rows past Nq / Nk arrive as zeros through the 3-D tensor maps. Padded queries, and
+  // queries that see no key, have Ls = -inf, so their P is 0. Padded keys of the last
+  // key tile need no mask: their dK and dV rows are not stored, and their dS meets
+  // zero rows of K in dQ = dS K. Ls and Dv are laid out per head with ntq * 128 rows.
+  // Causal masking is bottom-right aligned (query q sees keys k <= q + off): the first
+  // query tile whose last row sees key j * 128 is i_begin; the last query sees every
+  // key, so niter >= 1.
+  const int off = Nk - Nq;
+  const int first_q = j * kTile - (kTile - 1) - off;  // i_begin = ceil(first_q / 128)
+  const int i_begin =
+      !CAUSAL || first_q <= 0 ? 0 : (first_q + kTile - 1) / kTile;
+  const int niter = ntq - i_begin;
+  const long head_row = static_cast<long>(bh) * Nk;  // this key tile's head, in K rows
 
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -261,7 +269,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int st = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
         const int qtile = (i_begin + it) * kTile;  // first query row within the head
-        const long head_pad = static_cast<long>(bh) * ntiles * kTile;  // Ls / Dv rows
+        const long head_pad = static_cast<long>(bh) * ntq * kTile;  // Ls / Dv rows
         if (it >= 2 && !mbar_wait(bar(kBbQEmpty + st), (use - 1) & 1, abort_flag)) break;
         const uint32_t full = bar(kBbQFull + st);
         mbar_expect_tx(full, Lay::kTileBytes + 2 * 512);
@@ -391,7 +399,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int it = 0; it < niter && ok; ++it) {
       const int st = it & 1;
       const uint32_t ph = static_cast<uint32_t>(it & 1);
-      const bool diag = CAUSAL && (i_begin + it == j);
+      // causal: query column qc is masked for key row r when qc < r - dl
+      const int dl = (i_begin + it) * kTile + off - j * kTile;
+      const bool diag = CAUSAL && dl < kTile - 1;
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) &&
                           mbar_wait(bar(kBbSFull), ph, abort_flag));
@@ -434,7 +444,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (diag) {
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              if (half * 64 + q + e < r) p[q + e] = 0.f;
+              if (half * 64 + q + e < r - dl) p[q + e] = 0.f;
           }
         }
 #pragma unroll
@@ -489,7 +499,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       tc_fence_after();
       const long grow = head_row + static_cast<long>(j) * kTile + r;
-      const bool live_row = j * kTile + r < N;  // padded keys of the last tile are not stored
+      const bool live_row = j * kTile + r < Nk;  // padded keys of the last tile are not stored
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = (which == 0 ? Lay::tDV : Lay::tDK) + half * (D / 2);

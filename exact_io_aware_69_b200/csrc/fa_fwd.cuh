@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmOres, bool has_res,
-                  float* __restrict__ Lse, int N, float scale_log2) {
+                  float* __restrict__ Lse, int Nq, int Nk, float scale_log2) {
   using Lay = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -104,14 +104,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ntiles = (N + kTile - 1) / kTile;
-  const int bh = blockIdx.x / ntiles;
-  const int tr = blockIdx.x - bh * ntiles;
-  const int t = CAUSAL ? (ntiles - 1 - tr) : tr;  // heaviest causal tiles first
-  const int nkv = CAUSAL ? t + 1 : ntiles;
-  // Rows and keys of the last tile past N (when N % 128 != 0) come in as zeros from the
-  // 3-D tensor maps; the keys are masked below, the rows are not stored.
-  const int last_keys = N - (ntiles - 1) * kTile;  // valid keys in the last KV tile
+  const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head (one CTA each)
+  const int ntk = (Nk + kTile - 1) / kTile;  // key / value tiles per head
+  const int bh = blockIdx.x / ntq;
+  const int tr = blockIdx.x - bh * ntq;
+  const int t = CAUSAL ? (ntq - 1 - tr) : tr;  // heaviest causal tiles first
+  // Causal masking is bottom-right aligned: query q sees keys k <= q + off. The tile's
+  // last row sees keys up to kmax; tiles past it are never loaded. With Nq > Nk the
+  // first Nq - Nk queries see no key (O = 0, L = -inf); a tile of only such rows has
+  // nkv = 0.
+  const int off = Nk - Nq;
+  const int kmax = t * kTile + kTile - 1 + off;
+  const int nkv = !CAUSAL ? ntk : (kmax < 0 ? 0 : min(ntk, kmax / kTile + 1));
+  // Rows and keys of a last tile past Nq / Nk come in as zeros from the 3-D tensor
+  // maps; the keys are masked below, the rows are not stored.
+  const int last_keys = Nk - (ntk - 1) * kTile;  // valid keys in the last KV tile
 
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -265,11 +272,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         reg_fence32(sr + 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        // diagonal tile: key column > query row is masked; last tile: keys >= N
-        const bool diag = CAUSAL && j == t;
-        if (diag || (j == ntiles - 1 && last_keys < kTile)) {
-          int lim = (j == ntiles - 1 ? last_keys - 1 : kTile - 1) - half * 64;
-          if (diag) lim = min(lim, r - half * 64);
+        // causal: key column c is masked for row r when c > r + delta (the tiles
+        // along the diagonal band); last tile: keys >= Nk
+        const int delta = t * kTile + off - j * kTile;
+        const bool cmask = CAUSAL && delta < kTile - 1;
+        const bool kmask = j == ntk - 1 && last_keys < kTile;
+        if (cmask || kmask) {
+          int lim = kmask ? last_keys - 1 : kTile - 1;
+          if (cmask) lim = min(lim, r + delta);
+          lim -= half * 64;
 #pragma unroll
           for (int c = 0; c < 64; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
         }
@@ -283,10 +294,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (!ok) continue;
       const float cand = mx * scale_log2;
       const float m_new = (cand > m + kRescaleSlack) ? cand : m;
-      const float alpha = ex2_approx(m - m_new);  // 0 on the first tile, 1 if unchanged
+      // A row that sees no key keeps m = -inf: it takes alpha = 1 and subtracts 0, so
+      // that its p = 2^-inf = 0 and no inf - inf appears.
+      const bool empty_row = m_new == -INFINITY;
+      const float alpha = empty_row ? 1.f : ex2_approx(m - m_new);  // 0 on the first tile
       // pairs of lanes in packed fp32 (x2) arithmetic: argument, sums
       const uint64_t c2 = f2_pack(scale_log2, scale_log2);
-      const uint64_t nm2 = f2_pack(-m_new, -m_new);
+      const float m_sub = empty_row ? 0.f : m_new;
+      const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
       uint64_t sum2 = 0, sum2_o = 0;  // two packed +0.0f
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
@@ -341,9 +356,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (threadIdx.x == 0) FA_TRACE_EVENT(j, 7);
       m = m_new;
     }
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBarODone + ((nkv - 1) & 1)),
-                                                 static_cast<uint32_t>((nkv - 1) >> 1) & 1,
-                                                 abort_flag));
+    ok = __all_sync(0xffffffffu, ok && (nkv == 0 || mbar_wait(bar(kBarODone + ((nkv - 1) & 1)),
+                                                              static_cast<uint32_t>((nkv - 1) >> 1) & 1,
+                                                              abort_flag)));
     // both halves' sums: reuse the exchange buffer of parity (nkv & 1), which the pair
     // last used two tiles ago
     red[((nkv & 1) * 2 + half) * 128 + r] = l;
@@ -357,16 +372,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // further on, each in the 128-byte-swizzled layout of the tensor maps.
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l_o_row;
+      const float inv_l = l_o_row > 0.f ? 1.f / l_o_row : 0.f;  // rows that see no key: O = 0
       const uint32_t st_o = sbase + Lay::kK;
       const uint32_t st_r = st_o + Lay::kTileBytes;
       const int sw = r & 7;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + o_cols + c * 32, o);
-        tmem_wait_ld();
-        reg_fence32(o);
+        if (nkv > 0) {  // with no KV tile, O in TMEM was never written
+          tmem_ld32(lane_base + o_cols + c * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
         uint32_t hw[16], lw[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -395,8 +415,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       fence_async_smem();
-      if (half == 0 && t * kTile + r < N)
-        Lse[static_cast<long>(bh) * N + t * kTile + r] =
+      if (half == 0 && t * kTile + r < Nq)
+        Lse[static_cast<long>(bh) * Nq + t * kTile + r] =
             (m + log2f(l_row)) * 0.69314718055994530942f;
     }
     // all 256 softmax threads have staged their part (or all gave up together)

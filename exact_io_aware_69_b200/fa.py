@@ -28,9 +28,13 @@ _vp, _int, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_s
 SIGNATURES = {
     "fa_fwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32, _int,
                       _vp]),
+    "fa_fwd_qk": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _f32,
+                         _int, _vp]),
     "fa_bwd_workspace_size": (_sz, [_int, _int, _int, _int]),
     "fa_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
                       _int, _f32, _int, _vp, _sz, _vp]),
+    "fa_bwd_qk": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int,
+                         _int, _int, _int, _f32, _int, _vp, _sz, _vp]),
     "fa_bwd_preprocess": (_int, [_vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, _sz,
                                  _vp]),
     "fa_bwd_dkdv": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _f32,
@@ -103,17 +107,28 @@ def _ptr_or_none(t):
     return None if t is None else t.data_ptr()
 
 
+def _check_kv(q, k, v):
+    """k and v: [B, H, Nk, d] like q except for the sequence length."""
+    _check(k, "k")
+    _check(v, "v", k)
+    if k.dim() != 4 or k.shape[:2] != q.shape[:2] or k.shape[3] != q.shape[3] or \
+            k.dtype != q.dtype:
+        raise FaError(FA_ERR_INVALID, "k/v batch, heads, head dim or dtype differ from q")
+
+
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
             out_res=None, residual: bool = True, stream=None):
-    """(O, L, O_res) = attention(q, k, v) for [B, H, N, d] bf16/fp16 CUDA tensors.
+    """(O, L, O_res) = attention(q, k, v) for bf16/fp16 CUDA tensors, q [B, H, Nq, d],
+    k and v [B, H, Nk, d] (causal masking bottom-right aligned when Nq != Nk).
 
     O_res is the 16-bit rounding residual of O (None when residual=False); pass it to
     backward() so that D = rowsum(dO * O) is formed from O at near-fp32 precision."""
     import torch
     lib = load()
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, q)
+    _check(q, "q")
+    _check_kv(q, k, v)
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -122,11 +137,11 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
     if out_res is None and residual:
         out_res = torch.empty_like(q)
-    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                    _ptr_or_none(out_res), lse.data_ptr(), B, H, N, d, int(bool(causal)),
-                    float(scale), _dtype_code(q), _stream_handle(stream))
+    rc = lib.fa_fwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                       _ptr_or_none(out_res), lse.data_ptr(), B, H, N, Nk, d, int(bool(causal)),
+                       float(scale), _dtype_code(q), _stream_handle(stream))
     if rc != FA_OK:
-        raise FaError(rc, "fa_fwd")
+        raise FaError(rc, "fa_fwd_qk")
     return out, lse, out_res
 
 
@@ -140,25 +155,27 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale: float | None = No
     (o_res: the forward's rounding residual of O, or None)."""
     import torch
     lib = load()
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+    for t, n in ((q, "q"), (o, "o"), (do, "do")):
         _check(t, n, q)
+    _check_kv(q, k, v)
     _check(lse, "lse")
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     need = workspace_size(B, H, N, d)
     if workspace is None:
         workspace = torch.empty(max(need, 1), device=q.device, dtype=torch.uint8)
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    rc = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr_or_none(o_res),
-                    do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                    B, H, N, d,
-                    int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
-                    workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    rc = lib.fa_bwd_qk(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                       _ptr_or_none(o_res), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                       dk.data_ptr(), dv.data_ptr(), B, H, N, Nk, d, int(bool(causal)),
+                       float(scale), _dtype_code(q), workspace.data_ptr(),
+                       workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if rc != FA_OK:
-        raise FaError(rc, "fa_bwd")
+        raise FaError(rc, "fa_bwd_qk")
     return dq, dk, dv
 
 

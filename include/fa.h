@@ -80,6 +80,17 @@ int fa_fwd(const void *Q, const void *K, const void *V, void *O, void *O_res, fl
            int H, int N, int d, int causal, float scale, int dtype, void *stream);
 
 /*
+ * Forward with separate query and key lengths: Q, O, O_res [B][H][Nq][d], K, V
+ * [B][H][Nk][d], L [B][H][Nq]. Causal masking is bottom-right aligned: query i sees
+ * keys j <= i + Nk - Nq, so the last query sees every key (with Nq = Nk this is
+ * j <= i). With Nq > Nk the first Nq - Nk queries see no key; their O rows are 0
+ * and their L is -inf. Nk = 0 with Nq > 0 is FA_ERR_INVALID. fa_fwd is
+ * fa_fwd_qk(..., N, N, ...).
+ */
+int fa_fwd_qk(const void *Q, const void *K, const void *V, void *O, void *O_res, float *L, int B,
+              int H, int Nq, int Nk, int d, int causal, float scale, int dtype, void *stream);
+
+/*
  * Bytes of device workspace that fa_bwd needs for this shape: fp32 D and scaled L
  * ([B][H][Np] each, Np = N rounded up to a multiple of 128) plus an fp32 dQ
  * accumulator [B][H][N][d]: B*H*Np*8 + B*H*N*d*4. 0 for an empty problem;
@@ -99,6 +110,18 @@ int fa_bwd(const void *Q, const void *K, const void *V, const void *O, const voi
            const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H, int N,
            int d, int causal, float scale, int dtype, void *workspace, size_t workspace_bytes,
            void *stream);
+
+/*
+ * Backward with separate query and key lengths (shapes and masking as fa_fwd_qk; dQ
+ * and dO [B][H][Nq][d], dK and dV [B][H][Nk][d]). The workspace is sized by
+ * fa_bwd_workspace_size(B, H, Nq, d). Queries that see no key contribute nothing.
+ * With B*H*Nq == 0 and Nk > 0, dK and dV are set to zero (only they are touched).
+ * fa_bwd is fa_bwd_qk(..., N, N, ...).
+ */
+int fa_bwd_qk(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
+              const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H, int Nq,
+              int Nk, int d, int causal, float scale, int dtype, void *workspace,
+              size_t workspace_bytes, void *stream);
 
 /*
  * The three stages of fa_bwd, callable one by one (same arguments, same checks, same

@@ -34,7 +34,7 @@ def test_header_declares_the_boundary():
     assert names == sorted(["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_status",
                             "fa_status_string", "fa_version", "fa_bwd_preprocess",
                             "fa_bwd_dkdv", "fa_bwd_dq_convert", "fa_bwd_noalloc",
-                            "fa_selftest_wait_timeout"])
+                            "fa_selftest_wait_timeout", "fa_fwd_qk", "fa_bwd_qk"])
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -142,3 +142,24 @@ def test_workspace_size_pads_rows_per_head(lib, B, H, N, d):
     want = B * H * n_pad * 8 + B * H * N * d * 4
     assert lib.fa_bwd_workspace_size(B, H, N, d) == want
     assert (B * H * n_pad * 8) % 1024 == 0
+
+
+def _fwd_qk(lib, Nq, Nk, **kw):
+    a = dict(Q=P, K=P + 0x100000, V=P + 0x200000, O=P + 0x300000, R=None, L=P + 0x400000, B=1,
+             H=1, d=64, causal=1, scale=0.125, dtype=fa.FA_BF16)
+    a.update(kw)
+    return lib.fa_fwd_qk(a["Q"], a["K"], a["V"], a["O"], a["R"], a["L"], a["B"], a["H"], Nq, Nk,
+                         a["d"], a["causal"], a["scale"], a["dtype"], None)
+
+
+def test_qk_shapes_rejected_before_launch(lib):
+    """Nk = 0 with queries has no softmax; lengths are checked like N; Nq = 0 is empty."""
+    assert _fwd_qk(lib, 128, 0) == fa.FA_ERR_INVALID
+    assert _fwd_qk(lib, -1, 128) == fa.FA_ERR_INVALID
+    assert _fwd_qk(lib, 128, -5) == fa.FA_ERR_INVALID
+    assert _fwd_qk(lib, 128, 256, d=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd_qk(lib, 0, 256, Q=None, O=None, L=None) == fa.FA_OK
+    assert _fwd_qk(lib, 100, 1 << 30, B=4) == fa.FA_ERR_UNSUPPORTED  # 2^32 padded key rows
+    # no queries: the backward only zeroes dK and dV, which must then be valid
+    assert lib.fa_bwd_qk(None, None, None, None, None, None, None, None, None, None, 1, 1, 0,
+                         128, 64, 1, 0.125, fa.FA_BF16, None, 0, None) == fa.FA_ERR_INVALID
