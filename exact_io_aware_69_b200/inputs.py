@@ -141,6 +141,10 @@ WORKLOADS = {
     "c3": Workload("c3 B2 H32 N8192 d128 bf16 causal", 2, 32, 8192, 128, BF16, True, config_seed(3)),
     "c4": Workload("c4 B1 H16 N65536 d128 bf16 causal, 1% rows x8", 1, 16, 65536, 128, BF16, True,
                    config_seed(4), large_frac=0.01),
+    # c3 with a sequence length that is not a multiple of 128 (the last tile of every
+    # head is partial): the ragged-N path at the headline size
+    "c3r": Workload("c3r B2 H32 N8000 d128 bf16 causal", 2, 32, 8000, 128, BF16, True,
+                    config_seed(3, 1)),
 }
 
 
