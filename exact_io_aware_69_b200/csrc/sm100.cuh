@@ -392,27 +392,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// 2^x on the FMA/ALU pipes, without the MUFU unit (whose instructions share the
-// MIO issue queue with tcgen05.mma: a warp flooding it with ex2 starves the MMA
-// issuer on the same SM sub-partition). Cody-Waite style range reduction (Cody and
-// Waite, "Software Manual for the Elementary Functions", 1980): x = j + f with
-// j = round(x), obtained by adding 1.5 * 2^23 so that the low mantissa bits of the sum
-// hold j, and f = x - j in [-1/2, 1/2] exactly. 2^f comes from a degree-3 polynomial
-// whose coefficients were fitted for this kernel (weighted least squares on Chebyshev
-// nodes, minimising relative error: max 7.5e-5 on [-1/2, 1/2] in fp32 Horner form,
-// well below the 2^-9 / 2^-12 rounding of the 16-bit P it feeds); 2^j is added into
-// the exponent field: (bits of the shifted sum) << 23 equals j << 23 modulo 2^32.
-// Inputs below -125 are clamped (2^-125 is nothing next to a row sum >= 2^-8).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.05517161f, f, 0.24261111f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992806f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // Packed fp32 pairs (sm_100): one instruction for two lanes of arithmetic.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
