@@ -60,12 +60,14 @@ def _load():
                                        ctypes.c_double, dp, dp]
     lib.oracle_attn_bwd_qk.argtypes = [f64p, f64p, f64p, f64p, L_, L_, L_, L_, ctypes.c_int,
                                        ctypes.c_double, dp, dp, dp, dp, dp, dp]
+    lib.oracle_attn_window.argtypes = [f64p, f64p, f64p, dp, L_, L_, L_, L_, L_, L_,
+                                       ctypes.c_double, dp, dp, dp, dp, dp, dp]
     lib.oracle_attn_rows.argtypes = [f64p, f64p, f64p, dp, L_, L_, L_, ctypes.c_int,
                                      ctypes.c_double, L_, dp, dp, dp, dp, dp, dp]
     lib.oracle_attn_keys.argtypes = [f64p, f64p, f64p, f64p, L_, L_, L_, ctypes.c_int,
                                      ctypes.c_double, L_, dp, dp, dp, dp]
     for fn in ("oracle_attn_fwd", "oracle_attn_bwd", "oracle_attn_fwd_qk", "oracle_attn_bwd_qk",
-               "oracle_attn_rows", "oracle_attn_keys"):
+               "oracle_attn_rows", "oracle_attn_keys", "oracle_attn_window"):
         getattr(lib, fn).restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -183,3 +185,35 @@ def attn_keys(q, k, v, do, causal: bool, scale: float, bh_idx, key_idx):
                                 _ptr(bh_idx), _ptr(key_idx), _ptr(dk), _ptr(dv)),
            "oracle_attn_keys")
     return {"dk": dk, "dv": dv}
+
+
+def attn_window(q, k, v, do, window, scale: float):
+    """Attention with a (left, right) key window (negative = unbounded on that side):
+    query i sees keys j with i + Nk - Nq - left <= j <= i + Nk - Nq + right.
+    (-1, -1) is unmasked attention, (-1, 0) the bottom-right causal mask. ``do`` may be
+    None for the forward alone. Returns a dict like attn_bwd (gradients None without
+    ``do``)."""
+    lib = _load()
+    shp, kshp = q.shape, k.shape
+    BH, Nq, d = _shape(q)
+    Nk = _shape(k)[1]
+    wl, wr = (int(w) for w in window)
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    do = None if do is None else _f64(do)
+    out = {"o": np.empty((BH, Nq, d), np.float64), "L": np.empty((BH, Nq), np.float64)}
+    if do is not None:
+        out["dq"] = np.empty((BH, Nq, d), np.float64)
+        out["dk"] = np.empty((BH, Nk, d), np.float64)
+        out["dv"] = np.empty((BH, Nk, d), np.float64)
+        out["D"] = np.empty((BH, Nq), np.float64)
+    _check(lib.oracle_attn_window(q, k, v, _ptr(do), BH, Nq, Nk, d, wl, wr, float(scale),
+                                  _ptr(out["o"]), _ptr(out["L"]), _ptr(out.get("dq")),
+                                  _ptr(out.get("dk")), _ptr(out.get("dv")), _ptr(out.get("D"))),
+           "oracle_attn_window")
+    res = {"o": out["o"].reshape(shp), "L": out["L"].reshape(shp[:-1])}
+    if do is not None:
+        res.update(dq=out["dq"].reshape(shp), dk=out["dk"].reshape(kshp),
+                   dv=out["dv"].reshape(kshp), D=out["D"].reshape(shp[:-1]))
+    else:
+        res.update(dq=None, dk=None, dv=None, D=None)
+    return res

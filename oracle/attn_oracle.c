@@ -408,3 +408,117 @@ int oracle_attn_keys(const double *q, const double *k, const double *v, const do
     free(m); free(l); free(D); free(done);
     return err;
 }
+
+/*
+ * ----------------------------------------------------------------- windowed masks
+ * Local ("sliding window") attention: query i sees the keys j with
+ *     i + off - wl <= j <= i + off + wr,      off = Nk - Nq,
+ * clipped to [0, Nk), where a negative wl or wr leaves that side unbounded. So
+ * (wl, wr) = (-1, -1) is unmasked attention and (-1, 0) the bottom-right causal mask
+ * above. A row whose range is empty has O = 0, L = -inf, dQ = 0, D = 0. (Reading: the
+ * pages name combining the method with window attention as a use, without a
+ * definition; this is the usual left/right window.) These functions are separate from
+ * the ones above so that those stay as they are; they follow the same three steps over
+ * the row's key range [lo, hi).
+ */
+static void window_range(long i, long Nq, long Nk, long wl, long wr, long *lo, long *hi) {
+    const long c = i + (Nk - Nq);
+    long a = wl < 0 ? 0 : c - wl;
+    long b = wr < 0 ? Nk : c + wr + 1;
+    if (a < 0) a = 0;
+    if (b > Nk) b = Nk;
+    if (b < a) b = a;
+    *lo = a;
+    *hi = b;
+}
+
+/* One query row over keys [lo, hi): P_i (in p, indexed from lo), O_i, m_i, l_i and,
+ * with doi, D_i and dQ_i. */
+static void window_row(const double *qi, const double *kh, const double *vh, const double *doi,
+                       long lo, long hi, long d, double scale, double *p, double *dp,
+                       double *o_i, double *m_i, double *l_i, double *D_i, double *dq_i) {
+    const long n = hi - lo;
+    score_row(qi, kh + lo * d, n, d, scale, p);
+    softmax_row(p, n, m_i, l_i);
+    if (o_i) weighted_rows(p, vh + lo * d, n, d, o_i);
+    if (!doi) return;
+    double D = 0.0;
+    for (long j = 0; j < n; ++j) {
+        const double *vj = vh + (lo + j) * d;
+        double acc = 0.0;
+        for (long t = 0; t < d; ++t) acc += doi[t] * vj[t];
+        dp[j] = acc;
+        D += p[j] * acc;
+    }
+    *D_i = D;
+    if (dq_i) {
+        for (long j = 0; j < n; ++j) dp[j] = p[j] * (dp[j] - D);
+        weighted_rows(dp, kh + lo * d, n, d, dq_i);
+        for (long t = 0; t < d; ++t) dq_i[t] *= scale;
+    }
+}
+
+/* Forward and backward with a window (o, L, dq, dk, dv, D may each be NULL; dO may be
+ * NULL for the forward alone). Shapes as oracle_attn_bwd_qk. */
+int oracle_attn_window(const double *q, const double *k, const double *v, const double *dO,
+                       long BH, long Nq, long Nk, long d, long wl, long wr, double scale,
+                       double *o, double *L, double *dq, double *dk, double *dv, double *D_out) {
+    if (check_args(q, k, v, BH, Nq, Nk, d)) return ORC_EINVAL;
+    if ((dq || dk || dv || D_out) && !dO) return ORC_EINVAL;
+    if (Nq == 0 || Nk == 0 || BH == 0) return ORC_OK;
+    double *m = (double *)malloc(sizeof(double) * (size_t)Nq);
+    double *l = (double *)malloc(sizeof(double) * (size_t)Nq);
+    double *D = (double *)malloc(sizeof(double) * (size_t)Nq);
+    double *p = (double *)malloc(sizeof(double) * (size_t)Nk);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)Nk);
+    if (!m || !l || !D || !p || !dp) {
+        free(m); free(l); free(D); free(p); free(dp);
+        return ORC_ENOMEM;
+    }
+    for (long bh = 0; bh < BH; ++bh) {
+        const size_t hq = (size_t)bh * Nq * d, hk = (size_t)bh * Nk * d;
+        const double *qh = q + hq, *kh = k + hk, *vh = v + hk;
+        const double *doh = dO ? dO + hq : NULL;
+        for (long i = 0; i < Nq; ++i) {
+            long lo, hi;
+            window_range(i, Nq, Nk, wl, wr, &lo, &hi);
+            D[i] = 0.0;
+            window_row(qh + i * d, kh, vh, doh ? doh + i * d : NULL, lo, hi, d, scale, p, dp,
+                       o ? o + hq + (size_t)i * d : NULL, &m[i], &l[i], &D[i],
+                       dq ? dq + hq + (size_t)i * d : NULL);
+            if (L) L[(size_t)bh * Nq + i] = m[i] + log(l[i]);
+            if (D_out) D_out[(size_t)bh * Nq + i] = D[i];
+        }
+        if (!dk && !dv) continue;
+        /* dK_j, dV_j: the rows whose range holds key j */
+        for (long j = 0; j < Nk; ++j) {
+            double *gk = dk ? dk + hk + (size_t)j * d : NULL;
+            double *gv = dv ? dv + hk + (size_t)j * d : NULL;
+            for (long t = 0; t < d; ++t) {
+                if (gk) gk[t] = 0.0;
+                if (gv) gv[t] = 0.0;
+            }
+            const double *kj = kh + j * d, *vj = vh + j * d;
+            for (long i = 0; i < Nq; ++i) {
+                long lo, hi;
+                window_range(i, Nq, Nk, wl, wr, &lo, &hi);
+                if (j < lo || j >= hi) continue;
+                const double *qi = qh + i * d, *doi = doh + i * d;
+                double s = 0.0, dpv = 0.0;
+                for (long t = 0; t < d; ++t) {
+                    s += qi[t] * kj[t];
+                    dpv += doi[t] * vj[t];
+                }
+                s *= scale;
+                const double P = exp(s - m[i]) / l[i];
+                const double dS = P * (dpv - D[i]);
+                for (long t = 0; t < d; ++t) {
+                    if (gv) gv[t] += P * doi[t];
+                    if (gk) gk[t] += scale * dS * qi[t];
+                }
+            }
+        }
+    }
+    free(m); free(l); free(D); free(p); free(dp);
+    return ORC_OK;
+}

@@ -371,3 +371,72 @@ def test_queries_that_see_no_key(nq, nk):
         np.testing.assert_array_equal(got[name][:, e:], sq[name])
     for name in ("dk", "dv"):
         np.testing.assert_allclose(got[name], sq[name], rtol=1e-13, atol=1e-15)
+
+
+# ------------------------------------------------------------- key windows
+# (left, right) windows, the next mask variant. Pinned to the unmasked and causal
+# oracles, to a closed form, to single-query attention over the key slice, and to
+# central finite differences of the windowed forward.
+
+@pytest.mark.parametrize("nq,nk", [(6, 6), (4, 9), (9, 4)])
+def test_window_unbounded_and_causal_equal_the_plain_masks(nq, nk):
+    q, k, v, do = _qkv(nq, nk, 8, seed=300 + nq * 10 + nk)
+    for window, causal in (((-1, -1), False), ((-1, 0), True)):
+        got = oracle.attn_window(q, k, v, do, window, 0.4)
+        ref = oracle.attn_bwd(q, k, v, do, causal, 0.4)
+        for name in ("o", "L", "dq", "dk", "dv", "D"):
+            np.testing.assert_allclose(got[name], ref[name], rtol=1e-13, atol=1e-15,
+                                       err_msg=f"{name} window {window}")
+
+
+def test_window_of_one_key():
+    """(0, 0) with Nq = Nk: query i sees key i only, so O_i = v_i, L_i = s_ii, D_i =
+    dO_i . v_i, dV_i = dO_i and dQ = dK = 0 (P = 1, so dS = dP - D = 0)."""
+    q, k, v, do = _qkv(7, 7, 8, seed=17)
+    got = oracle.attn_window(q, k, v, do, (0, 0), 0.5)
+    np.testing.assert_array_equal(got["o"], v)
+    np.testing.assert_allclose(got["L"], 0.5 * np.einsum("bid,bid->bi", q, k), rtol=1e-14)
+    np.testing.assert_allclose(got["D"], np.einsum("bid,bid->bi", do, v), rtol=1e-14)
+    np.testing.assert_array_equal(got["dv"], do)
+    assert np.all(got["dq"] == 0) and np.all(got["dk"] == 0)
+
+
+@pytest.mark.parametrize("window", [(2, 1), (0, 3), (3, -1), (1, 0)])
+def test_window_rows_are_single_queries_over_the_slice(window):
+    nq, nk = 8, 11
+    q, k, v, _ = _qkv(nq, nk, 8, seed=41 + window[0] * 5 + window[1])
+    got = oracle.attn_window(q, k, v, None, window, 0.3)
+    off = nk - nq
+    for i in range(nq):
+        lo = 0 if window[0] < 0 else max(0, i + off - window[0])
+        hi = nk if window[1] < 0 else min(nk, i + off + window[1] + 1)
+        if hi <= lo:
+            assert np.all(got["o"][:, i] == 0) and np.all(got["L"][:, i] == -np.inf)
+            continue
+        o1, L1 = oracle.attn_fwd(q[:, i:i + 1], k[:, lo:hi], v[:, lo:hi], False, 0.3)
+        np.testing.assert_allclose(got["o"][:, i], o1[:, 0], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(got["L"][:, i], L1[:, 0], rtol=1e-13)
+
+
+def test_window_gradients_are_finite_differences():
+    """dQ, dK, dV of the windowed backward against central differences of
+    f = sum(O * dO) from the windowed forward."""
+    nq, nk, d, window, scale = 5, 7, 4, (2, 1), 0.45
+    q, k, v, do = _qkv(nq, nk, d, seed=77, bh=1)
+    got = oracle.attn_window(q, k, v, do, window, scale)
+
+    def f(qq, kk, vv):
+        return float(np.sum(oracle.attn_window(qq, kk, vv, None, window, scale)["o"] * do))
+
+    h = 1e-6
+    for name, arr in (("dq", q), ("dk", k), ("dv", v)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args = {"dq": (q, k, v), "dk": (q, k, v), "dv": (q, k, v)}[name]
+            a_p = [plus if x is arr else x for x in args]
+            a_m = [minus if x is arr else x for x in args]
+            num[idx] = (f(*a_p) - f(*a_m)) / (2 * h)
+        np.testing.assert_allclose(got[name], num, rtol=1e-6, atol=1e-8, err_msg=name)
