@@ -415,9 +415,10 @@ int oracle_attn_keys(const double *q, const double *k, const double *v, const do
  *     i + off - wl <= j <= i + off + wr,      off = Nk - Nq,
  * clipped to [0, Nk), where a negative wl or wr leaves that side unbounded. So
  * (wl, wr) = (-1, -1) is unmasked attention and (-1, 0) the bottom-right causal mask
- * above. A row whose range is empty has O = 0, L = -inf, dQ = 0, D = 0. (Reading: the
- * pages name combining the method with window attention as a use, without a
- * definition; this is the usual left/right window.) These functions are separate from
+ * above. A row whose range is empty has O = 0, L = -inf, dQ = 0, D = 0. (A reading:
+ * josueisai.com "flash-attention", section "Que ganas y que no", names window
+ * attention as what to combine the method with for very long sequences but does not
+ * define it; this is the usual left/right window.) These functions are separate from
  * the ones above so that those stay as they are; they follow the same three steps over
  * the row's key range [lo, hi).
  */
