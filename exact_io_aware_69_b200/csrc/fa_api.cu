@@ -223,35 +223,26 @@ struct BwdRun {
 };
 
 // ------------------------------------------------ backward without allocation
-// Scratch of fa_bwd_noalloc: a fixed device array that every GPU loading this
-// library holds until the process exits. 32 MiB covers the backward workspace of
-// B*H*N up to 64,527 rows at d = 128 (128,100 rows at d = 64).
+// Scratch of fa_bwd_noalloc: a fixed device array that every CUDA context using this
+// library holds until the context is destroyed. 32 MiB covers the backward workspace
+// of B*H*N up to 64,527 rows at d = 128 (127,100 rows at d = 64).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on the current device. Host code only sees a
-// host-side stand-in under that name, so the address is looked up once per device
-// (with that device current) and cached.
-constexpr int kMaxDevices = 64;
+// Device address of g_noalloc_scratch in the calling thread's current context. In
+// host code the array's name is only a host-side stand-in, and every context (the
+// primary one of each device, or one a host application created itself) holds its
+// own copy of the array at its own address, which also changes when a context is
+// destroyed and created again. So the address is looked up on every call, in the
+// context the work is enqueued in; the lookup is a host-side table query.
 void* noalloc_scratch_address(int* status) {
-  static void* addr[kMaxDevices] = {};
-  static std::mutex mu;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
     *status = FA_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
-      *status = FA_ERR_CUDA;
-      return nullptr;
-    }
-    addr[dev] = p;
-  }
   *status = FA_OK;
-  return addr[dev];
+  return p;
 }
 
 }  // namespace

@@ -155,16 +155,20 @@ int fa_bwd_dq_convert(void *dQ, int B, int H, int N, int d, float scale, int dty
  * calls no cudaMalloc, cudaFree or other allocating routine.
  *
  * Limit: fa_bwd_workspace_size(B, H, N, d) <= 32 MiB, i.e. (for N a multiple of 128)
- * B*H*N <= 64,527 at d = 128 and <= 128,100 at d = 64; larger problems return
+ * B*H*N <= 64,527 at d = 128 and <= 127,100 at d = 64 (each row takes 8 bytes of
+ * row statistics and 4*d bytes of dQ accumulator); larger problems return
  * FA_ERR_UNSUPPORTED before anything touches the device. Other checks and results
  * are those of fa_bwd.
  *
- * The first call on a device looks up the scratch array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that first
- * call before any stream capture. All calls on a device share the one array: the
- * part that must start at zero (the dQ accumulator) is cleared by every call, but
- * two calls whose work overlaps on the GPU (different streams, no ordering between
- * them) race on it and give wrong gradients. Order such calls on one stream.
+ * The array is per CUDA context: each context that runs this call (the primary
+ * context of a device, or one the host application created) holds its own copy.
+ * Every call looks up the array's address in the calling thread's current context
+ * (cudaGetSymbolAddress); the first call in a context may also load the library's
+ * device code there, so make that first call before any stream capture. All calls
+ * in one context share the one array: the part that must start at zero (the dQ
+ * accumulator) is cleared by every call, but two calls whose work overlaps on the
+ * GPU (different streams, no ordering between them) race on it and give wrong
+ * gradients. Order such calls on one stream.
  */
 int fa_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
                    const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H,

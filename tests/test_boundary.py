@@ -163,3 +163,18 @@ def test_qk_shapes_rejected_before_launch(lib):
     # no queries: the backward only zeroes dK and dV, which must then be valid
     assert lib.fa_bwd_qk(None, None, None, None, None, None, None, None, None, None, 1, 1, 0,
                          128, 64, 1, 0.125, fa.FA_BF16, None, 0, None) == fa.FA_ERR_INVALID
+
+
+def test_noalloc_scratch_limit_at_its_edge(lib):
+    """fa_bwd_noalloc's 32 MiB scratch: at d = 64 a row takes 8 + 256 bytes, so 992
+    tiles of 128 rows (126,976 rows) fit and 993 tiles (127,104 rows) do not; the
+    larger problem is refused before any pointer is used."""
+    limit = 32 << 20
+    assert lib.fa_bwd_workspace_size(1, 1, 126976, 64) <= limit
+    assert lib.fa_bwd_workspace_size(1, 1, 127104, 64) > limit
+    assert lib.fa_bwd_workspace_size(1, 1, 64512, 128) <= limit   # 504 tiles at d = 128
+    assert lib.fa_bwd_workspace_size(1, 1, 64640, 128) > limit
+    args = [P, P, P, P, None, P, P, P, P, P]
+    for B, H, N, d in ((1, 1, 127104, 64), (3, 1, 42368, 64), (1, 1, 64640, 128)):
+        assert lib.fa_bwd_noalloc(*args, B, H, N, d, 0, 0.125, fa.FA_BF16, None) == \
+            fa.FA_ERR_UNSUPPORTED
