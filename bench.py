@@ -36,7 +36,7 @@ if ROOT not in sys.path:
 
 import numpy as np  # noqa: E402
 
-from exact_io_aware_69_b200.inputs import WORKLOADS  # noqa: E402
+from exact_io_aware_69_b200.inputs import WORKLOADS, sweep_workloads  # noqa: E402
 
 METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16, causal/non) and % of tensor-core peak"
 UNIT = "TFLOP/s"
@@ -60,6 +60,8 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads, the small-call latency and the memory fit")
     return ap.parse_args()
 
 
@@ -190,6 +192,155 @@ def job_throughput(world, flops_per_rank_step, steps, max_ms):
     return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
 
 
+def torch_inputs(w, dev, seed):
+    """Seeded iid N(0,1) inputs of workload w drawn on the device, for the timing-only
+    runs: torch's generator, rounded to the 16-bit type; w's large-logit rows (floor(
+    frac * N) distinct rows per head, x8) are chosen with the same generator."""
+    import torch
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    shape = (w.B, w.H, w.N, w.d)
+    out = [torch.randn(shape, generator=g, device=dev, dtype=torch.float32) for _ in range(4)]
+    if w.large_frac > 0:
+        n_large = int(math.floor(w.large_frac * w.N))
+        qf = out[0].view(w.B * w.H, w.N, w.d)
+        for bh in range(w.B * w.H):
+            rows = torch.randperm(w.N, generator=g, device=dev)[:n_large]
+            qf[bh, rows] *= 8.0
+    return [t.to(tdt) for t in out]
+
+
+def time_workload(fa, w, dev, stream, steps, warmup, peak_burst):
+    """Device time per step of the forward and the three backward kernels of workload
+    w (CUDA events on the launching stream), and the rates they give."""
+    import torch
+    q, k, v, do = torch_inputs(w, dev, w.seed)
+    o, o_res = torch.empty_like(q), torch.empty_like(q)
+    L = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    dq, dk, dvv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+
+    def step(rec):
+        if rec:
+            ev[0].record(stream)
+        fa.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=L, out_res=o_res,
+                   stream=stream)
+        if rec:
+            ev[1].record(stream)
+        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=w.scale, o_res=o_res,
+                    workspace=ws, dq=dq, dk=dk, dv=dvv, stream=stream)
+        if rec:
+            ev[2].record(stream)
+
+    for _ in range(warmup):
+        step(False)
+    fwd_ms = bwd_ms = 0.0
+    for _ in range(steps):
+        step(True)
+        ev[2].synchronize()
+        fwd_ms += ev[0].elapsed_time(ev[1])
+        bwd_ms += ev[1].elapsed_time(ev[2])
+    st = fa.device_status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status {st} in {w.name}")
+    fwd_ms /= steps
+    bwd_ms /= steps
+    f, b = flops(w)
+    r = {"fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+         "fwd_tflops": round(f / fwd_ms / 1e9, 1), "bwd_tflops": round(b / bwd_ms / 1e9, 1),
+         "fwd_bwd_tflops_2p5x": round(2.5 * f / (fwd_ms + bwd_ms) / 1e9, 1),
+         "fwd_bwd_tflops_3p5x": round((f + b) / (fwd_ms + bwd_ms) / 1e9, 1)}
+    r["frac_3p5x_of_burst"] = round(r["fwd_bwd_tflops_3p5x"] / peak_burst, 3)
+    return r
+
+
+def small_call_latency(fa, dev, stream, iters=200):
+    """Config 1 (B1 H1 N256 d64): device time and host wall time of one forward +
+    backward through the binding, and the host cost of enqueueing each call."""
+    import torch
+    w = WORKLOADS["c1"]
+    q, k, v, do = torch_inputs(w, dev, w.seed)
+    o, o_res = torch.empty_like(q), torch.empty_like(q)
+    L = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    dq, dk, dvv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8)
+
+    def fwd():
+        fa.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=L, out_res=o_res,
+                   stream=stream)
+
+    def bwd():
+        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=w.scale, o_res=o_res,
+                    workspace=ws, dq=dq, dk=dk, dv=dvv, stream=stream)
+
+    for _ in range(20):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    e0.record(stream)
+    for _ in range(iters):
+        fwd()
+        bwd()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall = (time.perf_counter() - t0) / iters * 1e6
+    dev_us = e0.elapsed_time(e1) / iters * 1e3
+    enq_f, enq_b = [], []
+    for _ in range(50):
+        t = time.perf_counter()
+        fwd()
+        enq_f.append(time.perf_counter() - t)
+        t = time.perf_counter()
+        bwd()
+        enq_b.append(time.perf_counter() - t)
+        torch.cuda.synchronize()
+    return {"workload": "c1 B1 H1 N256 d64 bf16 non-causal", "iters": iters,
+            "device_us_per_fwd_bwd": round(dev_us, 2),
+            "host_wall_us_per_fwd_bwd": round(wall, 2),
+            "host_enqueue_us": {"forward": round(statistics.median(enq_f) * 1e6, 2),
+                                "backward": round(statistics.median(enq_b) * 1e6, 2)},
+            "note": "back-to-back calls through the Python binding; wall time includes the "
+                    "binding's marshalling and the C ABI's argument checks and tensor maps"}
+
+
+def linear_fit(xs, ys):
+    """Least squares y = a + b x: (slope b, intercept a, R^2)."""
+    x = np.asarray(xs, np.float64)
+    y = np.asarray(ys, np.float64)
+    b, a = np.polyfit(x, y, 1)
+    res = y - (a + b * x)
+    tot = y - y.mean()
+    return float(b), float(a), float(1.0 - (res @ res) / (tot @ tot))
+
+
+def peak_memory_vs_n(fa, dev, stream, ns=(1024, 2048, 4096, 8192, 16384, 32768, 65536)):
+    """Peak device memory of one forward + backward (inputs, outputs, workspace) at
+    B1 H16 d128 bf16 causal for each N, and a linear fit against N."""
+    import torch
+    peaks = []
+    for N in ns:
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        w = type(WORKLOADS["c4"])(f"mem N{N}", 1, 16, N, 128, "bf16", True, 7000 + N)
+        q, k, v, do = torch_inputs(w, dev, w.seed)
+        o, L, o_res = fa.forward(q, k, v, causal=True, scale=w.scale, stream=stream)
+        dq, dk, dvv = fa.backward(q, k, v, o, L, do, causal=True, scale=w.scale, o_res=o_res,
+                                  stream=stream)
+        torch.cuda.synchronize()
+        peaks.append(int(torch.cuda.max_memory_allocated() - base))
+        del q, k, v, do, o, L, o_res, dq, dk, dvv
+    slope, icpt, r2 = linear_fit(ns, peaks)
+    return {"shape": "B1 H16 d128 bf16 causal, fwd + bwd through the binding",
+            "N": list(ns), "peak_bytes": peaks, "slope_bytes_per_N": round(slope, 1),
+            "intercept_bytes": round(icpt, 1), "r2": r2}
+
+
 def run_reference(args, w, rank):
     """The oracle as it stands, timed on this host's cores (rank 0 only)."""
     if rank != 0:
@@ -246,21 +397,28 @@ def cpu_baseline_and_parity(w, inp, outs, target_s):
             got = outs[name].reshape(BH, N, d)[h].astype(np.float64)
             diff = np.abs(got - ref[name][0])
             rel = float((diff / np.maximum(1.0, np.abs(ref[name][0]))).max())
-            cur = worst.get(name, (0.0, 0.0))
-            worst[name] = (max(cur[0], rel), max(cur[1], float(diff.mean())))
+            cur = worst.get(name, (0.0, 0.0, 0.0))
+            worst[name] = (max(cur[0], float(diff.max())), max(cur[1], rel),
+                           max(cur[2], float(diff.mean())))
         dl = float(np.abs(outs["L"].reshape(BH, N)[h] - ref["L"][0]).max())
-        worst["L"] = (max(worst.get("L", (0.0, 0.0))[0], dl), 0.0)
+        worst["L"] = (max(worst.get("L", (0.0,))[0], dl), 0.0, 0.0)
     tol_max, tol_mean = (2e-2, 2e-3) if w.dtype == "bf16" else (5e-3, 5e-4)
-    ok = all(worst[n][0] <= tol_max and worst[n][1] <= tol_mean for n in ("o", "dq", "dk", "dv"))
+    # the literal max-abs bar; the relative reading (|got-ref|/max(1,|ref|)) only for the
+    # large-logit workload, whose x8 rows have gradients of magnitude ~10
+    relative = w.large_frac > 0
+    kmax = 1 if relative else 0
+    ok = all(worst[n][kmax] <= tol_max and worst[n][2] <= tol_mean for n in ("o", "dq", "dk", "dv"))
     ok = ok and worst["L"][0] <= 1e-3
     base = {"value": per_head * len(heads) / elapsed / 1e12, "unit": UNIT,
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{len(heads)} of {BH} heads (fwd+bwd, all {N} rows each), "
                       f"{elapsed:.1f} s of fp64 CPU work"}
     parity = {"heads_checked": heads, "ok": bool(ok),
-              "max_err": {n: round(worst[n][0], 6) for n in worst},
-              "mean_abs_err": {n: round(worst[n][1], 7) for n in ("o", "dq", "dk", "dv")},
-              "reading": "max |got-ref|/max(1,|ref|) vs 2e-2, mean |got-ref| vs 2e-3, L abs 1e-3"}
+              "max_abs_err": {n: round(worst[n][0], 6) for n in worst},
+              "max_rel_err": {n: round(worst[n][1], 6) for n in ("o", "dq", "dk", "dv")},
+              "mean_abs_err": {n: round(worst[n][2], 7) for n in ("o", "dq", "dk", "dv")},
+              "reading": ("max |got-ref|/max(1,|ref|)" if relative else "max |got-ref|")
+              + f" vs {tol_max:g}, mean |got-ref| vs {tol_mean:g}, L abs 1e-3"}
     return base, parity
 
 
@@ -384,12 +542,16 @@ def main():
               "fa_bwd_dq_kernel": rows * d * 4 + rows * d * 2}
     dom = max(per_kernel, key=per_kernel.get)
     dom_ms = per_kernel[dom] / steps
+    # The timed region is a fraction of a second at full clock, so the denominator is
+    # the burst peak (a kernel timed in a short loop); the sustained peak (seconds
+    # under the power cap) is printed beside it for reference.
     if dom in kflops:
         achieved = kflops[dom] / (dom_ms * 1e-3) / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_sus,
-                "unit": "TFLOP/s", "frac": achieved / peak_sus,
-                "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside the step loop)",
-                "frac_of_burst_peak": achieved / peak_burst,
+        roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": peak_burst,
+                "unit": "TFLOP/s", "frac": achieved / peak_burst,
+                "peak_kind": f"{peak_kind} bf16 burst (of measured cuBLAS; timed region "
+                             f"{total_ms:.0f} ms)",
+                "frac_of_sustained_peak": achieved / peak_sus,
                 "algorithmic_per_launch": kflops[dom], "avg_launch_ms": dom_ms}
     else:
         achieved = kbytes[dom] / (dom_ms * 1e-3) / 1e9
@@ -405,7 +567,7 @@ def main():
         e = {"avg_ms": ms, "share": per_kernel[n] / sum(per_kernel.values())}
         if n in kflops:
             e["tflops"] = kflops[n] / (ms * 1e-3) / 1e12
-            e["frac_of_sustained_peak"] = e["tflops"] / peak_sus
+            e["frac_of_burst_peak"] = e["tflops"] / peak_burst
         else:
             e["gbs"] = kbytes[n] / (ms * 1e-3) / 1e9
         kernels[n] = e
@@ -447,6 +609,20 @@ def main():
     e2e_ms = max_over_ranks([e2e_ms], pg, dev)[0]
     e2e_val = job_throughput(world, 2.5 * fwd_f, args.e2e_steps, e2e_ms)
 
+    extras = {}
+    if rank == 0 and not args.no_extras:
+        # the metric's other named workloads (fwd and fwd+bwd, causal and not, fp16, d=64)
+        by_w = {}
+        for name in ("c2", "c2c", "c4"):
+            by_w[WORKLOADS[name].name] = time_workload(fa, WORKLOADS[name], dev, stream, 5, 3,
+                                                       peak_burst)
+        for sw in sweep_workloads():
+            by_w[sw.name] = time_workload(fa, sw, dev, stream, 5, 3, peak_burst)
+        extras["by_workload"] = by_w
+        extras["latency_small"] = small_call_latency(fa, dev, stream)
+        extras["peak_memory"] = peak_memory_vs_n(fa, dev, stream)
+        torch.cuda.empty_cache()
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -455,10 +631,11 @@ def main():
         "fwd_tflops": fwd_f / (fwd_ms * 1e-3) / 1e12,
         "bwd_tflops": bwd_f / (bwd_ms * 1e-3) / 1e12,
         "fwd_bwd_tflops_3p5x": job_throughput(world, fwd_f + bwd_f, steps, total_ms),
-        "pct_of_peak": {"fwd": fwd_f / (fwd_ms * 1e-3) / 1e12 / peak_sus,
-                        "fwd_bwd_2p5x": value / world / peak_sus,
-                        "fwd_bwd_3p5x": (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12 / peak_sus,
-                        "peak": peak_sus, "peak_kind": f"{peak_kind} bf16 sustained"},
+        "pct_of_peak": {"fwd": fwd_f / (fwd_ms * 1e-3) / 1e12 / peak_burst,
+                        "fwd_bwd_2p5x": value / world / peak_burst,
+                        "fwd_bwd_3p5x": (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12 / peak_burst,
+                        "peak": peak_burst, "peak_kind": f"{peak_kind} bf16 burst",
+                        "sustained_peak": peak_sus},
         "kernels": kernels,
         "roofline": roof,
         "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -467,6 +644,7 @@ def main():
         "gpu_launches": 4 * steps,
         "clocks": clocks,
     }
+    line.update(extras)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         outs = {"o": o.float().cpu().numpy(), "dq": dq.float().cpu().numpy(),

@@ -27,27 +27,33 @@ def to_f64(t) -> np.ndarray:
 
 
 def errors(got: np.ndarray, ref: np.ndarray):
-    """(max of |got - ref| / max(1, |ref|), mean of |got - ref|).
-
-    The max-abs bar is read as absolute where |ref| <= 1 and relative above: a 16-bit
-    value of magnitude m carries a rounding error of up to m * 2^-9 (bf16) or m * 2^-12
-    (fp16) however exactly it is computed, so for gradients of magnitude ~10 (the
-    large-logit rows) no 16-bit result can be within 2e-2 absolute.
-    test_tolerance_floor.py shows this on the exact bf16-operand pipeline.
-    """
+    """(max |got - ref|, max |got - ref| / max(1, |ref|), mean |got - ref|)."""
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
     diff = np.abs(got - ref)
-    return float((diff / np.maximum(1.0, np.abs(ref))).max()), float(diff.mean())
+    return (float(diff.max()), float((diff / np.maximum(1.0, np.abs(ref))).max()),
+            float(diff.mean()))
 
 
-def assert_close(name: str, got, ref, dtype: str):
-    mx, mean = errors(got, ref)
+def assert_close(name: str, got, ref, dtype: str, relative: bool = False):
+    """Hold `got` to the parity bar: max-abs and mean-abs of |got - ref|.
+
+    The max bar is the literal absolute one unless `relative` is set. Only the
+    large-logit workloads set it: there the max bar is read as absolute where
+    |ref| <= 1 and relative above, because a 16-bit value of magnitude m carries a
+    rounding error of up to m * 2^-9 (bf16) or m * 2^-12 (fp16) however exactly it is
+    computed, and the gradients of the x8 rows reach |dK| ~ 10-16, where no 16-bit
+    result can be within 2e-2 absolute (test_tolerance_floor.py shows this on the
+    exact bf16-operand pipeline). Mean-abs is always absolute.
+    """
+    abs_max, rel_max, mean = errors(got, ref)
     tmax, tmean = TOL[dtype]
     assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    mx = rel_max if relative else abs_max
     assert mx <= tmax and mean <= tmean, (
-        f"{name}: max-abs {mx:.3e} (tol {tmax:.0e}), mean-abs {mean:.3e} (tol {tmean:.0e})")
-    return mx, mean
+        f"{name}: max-abs {abs_max:.3e}, max-rel {rel_max:.3e} ({'relative' if relative else 'absolute'}"
+        f" bar {tmax:.0e}), mean-abs {mean:.3e} (tol {tmean:.0e})")
+    return abs_max, rel_max, mean
 
 
 def assert_close_L(got, ref):

@@ -63,3 +63,23 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["metric"] == bench.METRIC
+
+
+def test_linear_fit_recovers_slope_and_r2():
+    slope, icpt, r2 = bench.linear_fit([1, 2, 4, 8], [13, 23, 43, 83])
+    assert slope == pytest.approx(10.0) and icpt == pytest.approx(3.0) and r2 == pytest.approx(1.0)
+    _, _, r2 = bench.linear_fit([1, 2, 3, 4], [1, 4, 9, 16])
+    assert r2 < 1.0
+
+
+def test_timing_inputs_have_the_workload_structure():
+    """Seeded device-drawn inputs (timing runs): shape, dtype, and exactly floor(0.01 N)
+    rows per head scaled x8 for the large-logit workload."""
+    import torch
+    w = type(bench.WORKLOADS["c4"])("t", 1, 2, 1000, 64, "bf16", True, 5, large_frac=0.01)
+    q, k, v, do = bench.torch_inputs(w, "cpu", 5)
+    assert q.shape == (1, 2, 1000, 64) and q.dtype == torch.bfloat16
+    q2, _, _, _ = bench.torch_inputs(w, "cpu", 5)
+    assert torch.equal(q, q2)
+    norms = q.float().norm(dim=-1)[0]             # [H, N]
+    assert ((norms > 40).sum(dim=1) == 10).all()  # ~8 * sqrt(64) vs ~sqrt(64)

@@ -178,3 +178,17 @@ def test_noalloc_scratch_limit_at_its_edge(lib):
     for B, H, N, d in ((1, 1, 127104, 64), (3, 1, 42368, 64), (1, 1, 64640, 128)):
         assert lib.fa_bwd_noalloc(*args, B, H, N, d, 0, 0.125, fa.FA_BF16, None) == \
             fa.FA_ERR_UNSUPPORTED
+
+
+def test_register_split_kernels_compiled_with_their_launch_budget():
+    """fa_bwd_main_kernel's setmaxnreg split (2 x 128 + 200 + 56 per sub-partition)
+    assumes exactly 128 registers per thread at launch; the build fails otherwise, and
+    ptxas's report of this build must show it for every instantiation."""
+    rep = build.resources()
+    mains = {k: v for k, v in rep.items() if "fa_bwd_main_kernel" in k}
+    assert len(mains) == 8  # d in {64, 128} x causal x dtype
+    assert all(v["registers"] == 128 for v in mains.values()), mains
+    with pytest.raises(RuntimeError):
+        build.check_resources({"_ZN2fa18fa_bwd_main_kernelILi64E": {"registers": 120,
+                                                                   "spill_stores": 0,
+                                                                   "spill_loads": 0}})

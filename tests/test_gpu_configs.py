@@ -43,12 +43,17 @@ def _head(inp, w, h):
     return [inp.wide[n][h:h + 1].astype(np.float64) for n in ("q", "k", "v", "do")]
 
 
+def _relative(w):
+    """The relative reading of the max bar applies to the large-logit workload only."""
+    return w.large_frac > 0
+
+
 def _check_heads(w, inp, got, heads):
     for h in heads:
         ref = oracle.attn_bwd(*_head(inp, w, h), w.causal, w.scale)
         assert_close_L(got["L"][h], ref["L"][0])
         for n in ("o", "dq", "dk", "dv"):
-            assert_close(f"{n}[head {h}]", got[n][h], ref[n][0], w.dtype)
+            assert_close(f"{n}[head {h}]", got[n][h], ref[n][0], w.dtype, _relative(w))
 
 
 def _check_rows(w, inp, got, heads, rows_per_head, rng, extra_rows=None):
@@ -60,16 +65,30 @@ def _check_rows(w, inp, got, heads, rows_per_head, rng, extra_rows=None):
         rows = np.array(sorted(rows))
         ref = oracle.attn_rows(*_head(inp, w, h), w.causal, w.scale, np.zeros(len(rows)), rows)
         assert_close_L(got["L"][h, rows], ref["L"])
-        assert_close(f"o[head {h}]", got["o"][h, rows], ref["o"], w.dtype)
-        assert_close(f"dq[head {h}]", got["dq"][h, rows], ref["dq"], w.dtype)
+        assert_close(f"o[head {h}]", got["o"][h, rows], ref["o"], w.dtype, _relative(w))
+        assert_close(f"dq[head {h}]", got["dq"][h, rows], ref["dq"], w.dtype, _relative(w))
 
 
 def _check_keys(w, inp, got, heads, keys):
     keys = np.array(sorted(set(int(x) for x in keys)))
     for h in heads:
         ref = oracle.attn_keys(*_head(inp, w, h), w.causal, w.scale, np.zeros(len(keys)), keys)
-        assert_close(f"dk[head {h}]", got["dk"][h, keys], ref["dk"], w.dtype)
-        assert_close(f"dv[head {h}]", got["dv"][h, keys], ref["dv"], w.dtype)
+        assert_close(f"dk[head {h}]", got["dk"][h, keys], ref["dk"], w.dtype, _relative(w))
+        assert_close(f"dv[head {h}]", got["dv"][h, keys], ref["dv"], w.dtype, _relative(w))
+
+
+def _heavy_keys(w, inp, h, count):
+    """The keys that the scaled-up (large-logit) query rows of head h weight most: for
+    each such row its highest-scoring visible key, ranked by that key's probability
+    (numpy on the 16-bit inputs; a row's probabilities need only its own scores)."""
+    q, k = inp.wide["q"][h].astype(np.float64), inp.wide["k"][h].astype(np.float64)
+    best = []
+    for i in np.sort(inp.large_rows[h]):
+        s = (k[:i + 1] @ q[i]) * w.scale if w.causal else (k @ q[i]) * w.scale
+        j = int(np.argmax(s))
+        best.append((float(1.0 / np.exp(s - s[j]).sum()), j))
+    best.sort(reverse=True)
+    return [j for _, j in best[:count]]
 
 
 def _check_identities(w, inp, got):
@@ -127,8 +146,13 @@ def test_config4_long_context_large_logits():
     BH = w.B * w.H
     rng = np.random.default_rng(4)
     _check_rows(w, inp, got, range(BH), 6, rng, extra_rows=inp.large_rows)
-    # keys of the last tiles need only the rows behind them
-    _check_keys(w, inp, got, [0, BH - 1], list(range(w.N - 130, w.N)) + [w.N - 1000])
+    # head 0: key tile 0 (the CTA with the longest loop: every query tile sees it), the
+    # keys that the x8 rows weight most, and the last keys; one pass of the oracle's
+    # row statistics over the whole head serves all of them
+    heavy = _heavy_keys(w, inp, 0, 16)
+    _check_keys(w, inp, got, [0], list(range(128)) + heavy + list(range(w.N - 130, w.N)))
+    # last head: keys of the last tiles, which need only the rows behind them
+    _check_keys(w, inp, got, [BH - 1], list(range(w.N - 130, w.N)) + [w.N - 1000])
     _check_identities(w, inp, got)
 
 

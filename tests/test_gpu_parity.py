@@ -78,7 +78,7 @@ def test_large_logit_rows(causal):
     _, got, ref = _run(1, 2, 512, 128, BF16, causal, seed=4242, large_frac=0.05)
     assert_close_L(to_f64(got["L"]), ref["L"])
     for name in ("o", "dq", "dk", "dv"):
-        assert_close(name, to_f64(got[name]), ref[name], BF16)
+        assert_close(name, to_f64(got[name]), ref[name], BF16, relative=True)
 
 
 def test_repeat_runs_are_stable():
