@@ -440,3 +440,55 @@ def test_window_gradients_are_finite_differences():
             a_m = [minus if x is arr else x for x in args]
             num[idx] = (f(*a_p) - f(*a_m)) / (2 * h)
         np.testing.assert_allclose(got[name], num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+# ---------------------------------------------------------------- split and merge
+@pytest.mark.parametrize("nq", [1, 4, 16])
+@pytest.mark.parametrize("nk", [1, 37, 300])
+@pytest.mark.parametrize("window", [(-1, -1), (-1, 0), (20, 3), (0, 0)])
+def test_split_keys_then_merge_equals_the_definition(nq, nk, window):
+    """Cutting the keys into blocks, attending within each block and merging the
+    blocks' (o, L) by their log-sum-exps gives the plain definition back (decode's
+    split-KV path), for every split, including blocks in which a row sees no key."""
+    from oracle.recurrence import attn_fwd_split, random_split
+    rng = np.random.default_rng(nq * 1000 + nk)
+    d = 8
+    q = rng.standard_normal((nq, d))
+    k = rng.standard_normal((nk, d))
+    v = rng.standard_normal((nk, d))
+    ref = oracle.attn_window(q[None], k[None], v[None], None, window, 0.7)
+    for _ in range(3):
+        O, L = attn_fwd_split(q, k, v, window, 0.7, random_split(nk, rng))
+        empty = np.isneginf(ref["L"][0])
+        assert np.array_equal(np.isneginf(L), empty)
+        np.testing.assert_allclose(L[~empty], ref["L"][0][~empty], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(O, ref["o"][0], rtol=0, atol=1e-12)
+
+
+def test_merge_is_order_free_and_ignores_empty_blocks():
+    from oracle.recurrence import merge_partials
+    rng = np.random.default_rng(7)
+    o = rng.standard_normal((5, 4))
+    L = rng.standard_normal(5) * 10
+    o1, L1 = merge_partials(o, L)
+    perm = rng.permutation(5)
+    o2, L2 = merge_partials(o[perm], L[perm])
+    np.testing.assert_allclose(o2, o1, atol=1e-13)
+    assert abs(L2 - L1) < 1e-13
+    # merging two merged groups = merging all at once (the merge is associative)
+    oa, La = merge_partials(o[:2], L[:2])
+    ob, Lb = merge_partials(o[2:], L[2:])
+    o3, L3 = merge_partials([oa, ob], [La, Lb])
+    np.testing.assert_allclose(o3, o1, atol=1e-13)
+    assert abs(L3 - L1) < 1e-13
+    # an extra block with no visible key (L = -inf, any o) changes nothing
+    o4, L4 = merge_partials(np.vstack([o, np.full((1, 4), 1e30)]), np.append(L, -np.inf))
+    np.testing.assert_allclose(o4, o1, atol=1e-13)
+    assert L4 == L1
+    # no block saw a key: O = 0, L = -inf
+    o5, L5 = merge_partials(np.ones((2, 4)), [-np.inf, -np.inf])
+    assert np.all(o5 == 0) and L5 == -np.inf
+    # closed form for two equal blocks: L = L_s + ln 2, o = mean of the two outputs
+    o6, L6 = merge_partials(o[:2], [1.5, 1.5])
+    np.testing.assert_allclose(o6, o[:2].mean(axis=0), atol=1e-14)
+    assert abs(L6 - (1.5 + math.log(2))) < 1e-14
