@@ -211,26 +211,42 @@ def torch_inputs(w, dev, seed):
     return [t.to(tdt) for t in out]
 
 
-def time_workload(fa, w, dev, stream, steps, warmup, peak_burst):
+def visible_pairs(Nq, Nk, window):
+    """(query, key) pairs inside the (left, right) key window (negative = unbounded),
+    bottom-right aligned: the algorithmic FLOP count of a windowed pass is 4 d per pair
+    forward."""
+    off = Nk - Nq
+    i = np.arange(Nq, dtype=np.int64)
+    lo = np.zeros(Nq, np.int64) if window[0] < 0 else np.maximum(0, i + off - window[0])
+    hi = np.full(Nq, Nk - 1, np.int64) if window[1] < 0 else np.minimum(Nk - 1, i + off + window[1])
+    return int(np.maximum(0, hi - lo + 1).sum())
+
+
+def time_workload(fa, w, dev, stream, steps, warmup, peak_burst, window=None, layout="bhnd",
+                  deterministic=False):
     """Device time per step of the forward and the three backward kernels of workload
-    w (CUDA events on the launching stream), and the rates they give."""
+    w (CUDA events on the launching stream), and the rates they give. `window`
+    replaces w's causal flag by a key window (FLOPs counted over the visible pairs)."""
     import torch
     q, k, v, do = torch_inputs(w, dev, w.seed)
+    if layout == "bnhd":
+        q, k, v, do = (t.transpose(1, 2).contiguous() for t in (q, k, v, do))
     o, o_res = torch.empty_like(q), torch.empty_like(q)
     L = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
     dq, dk, dvv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8)
+    ws = torch.empty(fa.workspace_size(w.B, w.H, w.N, w.d, deterministic=deterministic),
+                     device=dev, dtype=torch.uint8)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    mask = dict(causal=w.causal, window=window, layout=layout)
 
     def step(rec):
         if rec:
             ev[0].record(stream)
-        fa.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=L, out_res=o_res,
-                   stream=stream)
+        fa.forward(q, k, v, scale=w.scale, out=o, lse=L, out_res=o_res, stream=stream, **mask)
         if rec:
             ev[1].record(stream)
-        fa.backward(q, k, v, o, L, do, causal=w.causal, scale=w.scale, o_res=o_res,
-                    workspace=ws, dq=dq, dk=dk, dv=dvv, stream=stream)
+        fa.backward(q, k, v, o, L, do, scale=w.scale, o_res=o_res, workspace=ws, dq=dq, dk=dk,
+                    dv=dvv, stream=stream, deterministic=deterministic, **mask)
         if rec:
             ev[2].record(stream)
 
@@ -248,12 +264,49 @@ def time_workload(fa, w, dev, stream, steps, warmup, peak_burst):
     fwd_ms /= steps
     bwd_ms /= steps
     f, b = flops(w)
+    if window is not None:
+        f = 4.0 * w.B * w.H * w.d * visible_pairs(w.N, w.N, window)
+        b = 2.5 * f
     r = {"fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
          "fwd_tflops": round(f / fwd_ms / 1e9, 1), "bwd_tflops": round(b / bwd_ms / 1e9, 1),
          "fwd_bwd_tflops_2p5x": round(2.5 * f / (fwd_ms + bwd_ms) / 1e9, 1),
          "fwd_bwd_tflops_3p5x": round((f + b) / (fwd_ms + bwd_ms) / 1e9, 1)}
     r["frac_3p5x_of_burst"] = round(r["fwd_bwd_tflops_3p5x"] / peak_burst, 3)
     return r
+
+
+def time_decode(fa, B, H, Nq, Nk, d, dev, stream, steps, warmup, hbm_peak):
+    """The split-KV decode path: Nq rows per head against Nk keys, causal. Its bound is
+    HBM: K and V are read once (plus Q, O, L), so the rate is reported in GB/s."""
+    import torch
+    w = type(WORKLOADS["c4"])(f"decode Nq{Nq} Nk{Nk}", B, H, Nk, d, "bf16", True, 9000 + Nq)
+    _, k, v, _ = torch_inputs(w, dev, w.seed)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 1)
+    q = torch.randn((B, H, Nq, d), generator=g, device=dev).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    L = torch.empty((B, H, Nq), device=dev, dtype=torch.float32)
+    need = int(fa.load().fa_decode_workspace_size(B, H, Nq, Nk, d, -1, 0))
+    ws = torch.empty(max(need, 1), device=dev, dtype=torch.uint8)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        fa.decode(q, k, v, causal=True, out=o, lse=L, workspace=ws, stream=stream)
+    e0.record(stream)
+    for _ in range(steps):
+        fa.decode(q, k, v, causal=True, out=o, lse=L, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st = fa.device_status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status {st} in decode")
+    ms = e0.elapsed_time(e1) / steps
+    kv_bytes = 2 * B * H * Nk * d * 2
+    all_bytes = kv_bytes + 2 * B * H * Nq * d * 2 + B * H * Nq * 4
+    flops_ = 4.0 * B * H * d * visible_pairs(Nq, Nk, (-1, 0))
+    return {"shape": f"B{B} H{H} Nq{Nq} Nk{Nk} d{d} bf16 causal", "ms": round(ms, 4),
+            "kv_gbs": round(kv_bytes / ms / 1e6, 1), "hbm_gbs": round(all_bytes / ms / 1e6, 1),
+            "frac_of_hbm_peak": round(all_bytes / ms / 1e6 / hbm_peak, 3),
+            "tflops": round(flops_ / ms / 1e9, 2), "splits_workspace_bytes": need}
 
 
 def small_call_latency(fa, dev, stream, iters=200):
@@ -618,7 +671,18 @@ def main():
                                                        peak_burst)
         for sw in sweep_workloads():
             by_w[sw.name] = time_workload(fa, sw, dev, stream, 5, 3, peak_burst)
+        # the rows beyond the basic calls, on the headline shape
+        c3 = WORKLOADS["c3"]
+        by_w["c3 sliding window (1024, 0)"] = time_workload(fa, c3, dev, stream, 5, 3, peak_burst,
+                                                            window=(1024, 0))
+        by_w["c3 [B,N,H,d] layout"] = time_workload(fa, c3, dev, stream, 5, 3, peak_burst,
+                                                    layout="bnhd")
+        by_w["c3 deterministic backward"] = time_workload(fa, c3, dev, stream, 5, 3, peak_burst,
+                                                          deterministic=True)
         extras["by_workload"] = by_w
+        hbm = float(peaks["hbm_gbs"])
+        extras["decode"] = [time_decode(fa, 4, 32, nq, 65536, 128, dev, stream, 10, 3, hbm)
+                            for nq in (1, 4, 16)]
         extras["latency_small"] = small_call_latency(fa, dev, stream)
         extras["peak_memory"] = peak_memory_vs_n(fa, dev, stream)
         torch.cuda.empty_cache()

@@ -8,7 +8,10 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_band.cuh"
 #include "fa_bwd.cuh"
+#include "fa_bwd_dq.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 
 namespace fa {
@@ -29,8 +32,10 @@ __global__ void fa_selftest_wait_kernel(long long limit_cycles) {
 
 namespace {
 
-constexpr int kVersion = 1;
+constexpr int kVersion = 2;
 constexpr size_t kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+// Nq + Nk must stay below this so that no window arithmetic overflows 32 bits.
+constexpr long long kMaxRowsPerHead = 1LL << 29;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -51,45 +56,60 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH][N][d] row-major tensor seen in three dimensions (column, row within a head,
-// head), so that a 128-row box reaching past a head's N reads zeros and writes
-// nothing there. 16-bit: box of 64 columns x 128 rows; fp32 (the dQ accumulator,
-// target of TMA reduce-adds): 32 columns (128 bytes) x 128 rows. 128-byte swizzle.
-bool make_tmap3(CUtensorMap* map, const void* ptr, int BH, int N, int d,
+// Element strides (b, h, n) of a [B][H][N][d] or [B][N][H][d] tensor.
+fa::Strides strides_of(int layout, int H, int N, int d) {
+  const long D = d;
+  if (layout == FA_LAYOUT_BNHD) return {static_cast<long>(N) * H * D, D, static_cast<long>(H) * D};
+  return {static_cast<long>(H) * N * D, static_cast<long>(N) * D, D};
+}
+
+// A tensor seen in four dimensions (column, row within a head, head, batch) with the
+// strides of its layout, so that a 128-row box reaching past a head's N reads zeros
+// and writes nothing there. 16-bit: box of 64 columns x 128 rows; fp32 (the dQ
+// accumulator, target of TMA reduce-adds): 32 columns (128 bytes) x 128 rows.
+// 128-byte swizzle.
+bool make_tmap4(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, int layout,
                 CUtensorMapDataType type, int esize) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
-                        static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esize,
-                           static_cast<cuuint64_t>(N) * d * esize};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  const fa::Strides s = strides_of(layout, H, N, d);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.sn) * esize,
+                           static_cast<cuuint64_t>(s.sh) * esize,
+                           static_cast<cuuint64_t>(s.sb) * esize};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / esize), 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, type, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
-bool make_tmap(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype) {
-  return make_tmap3(map, ptr, BH, N, d,
+bool make_tmap(CUtensorMap* map, const void* ptr, int B, int H, int N, int d, int layout,
+               int dtype) {
+  return make_tmap4(map, ptr, B, H, N, d, layout,
                     dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                     2);
 }
-bool make_tmap_f32(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
-  return make_tmap3(map, ptr, BH, N, d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+// The dQ accumulator is the library's own [B][H][N][d] fp32 array.
+bool make_tmap_f32(CUtensorMap* map, const void* ptr, int B, int H, int N, int d) {
+  return make_tmap4(map, ptr, B, H, N, d, FA_LAYOUT_BHND, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p && aligned16(p); }
 
-// Shape checks shared by the forward and backward entry points. Returns FA_OK to
-// proceed, or an error; *empty is set for a valid problem with no query rows (the
-// backward then still owes dK = dV = 0 when Nk > 0). Keys are required when there are
-// queries: a row with no key at all has no softmax.
-int check_shape_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale, bool* empty) {
+// Shape checks shared by every entry point. Returns FA_OK to proceed, or an error;
+// *empty is set for a valid problem with no query rows (the backward then still owes
+// dK = dV = 0 when Nk > 0). Keys are required when there are queries: a row with no
+// key at all has no softmax.
+int check_shape(int B, int H, int Nq, int Nk, int d, int layout, int dtype, float scale,
+                bool* empty) {
   *empty = false;
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return FA_ERR_INVALID;
   if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * Nq == 0) {
@@ -97,6 +117,7 @@ int check_shape_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale, 
     return FA_OK;
   }
   if (Nk == 0) return FA_ERR_INVALID;
+  if (static_cast<long long>(Nq) + Nk > kMaxRowsPerHead) return FA_ERR_UNSUPPORTED;
   // TMA coordinates and grid indices are 32-bit (rows counted with N padded to 128)
   const long long pq = (Nq + fa::kTile - 1) / fa::kTile * fa::kTile;
   const long long pk = (Nk + fa::kTile - 1) / fa::kTile * fa::kTile;
@@ -104,25 +125,38 @@ int check_shape_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale, 
     return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
-int check_shape(int B, int H, int N, int d, int dtype, float scale, bool* empty) {
-  return check_shape_qk(B, H, N, N, d, dtype, scale, empty);
+
+// The key window in the kernels' form: an edge that bounds nothing becomes
+// fa::kUnbounded; *band is false when no (query, key) pair is outside the window.
+struct Window {
+  int wl, wr;
+  bool band;
+};
+Window window_of(int Nq, int Nk, int left, int right) {
+  Window w;
+  w.wl = (left < 0 || left >= fa::kUnbounded) ? fa::kUnbounded : left;
+  w.wr = (right < 0 || right >= fa::kUnbounded) ? fa::kUnbounded : right;
+  // every key is visible iff the left edge reaches key 0 from the last query and the
+  // right edge reaches key Nk - 1 from the first
+  w.band = !(static_cast<long long>(w.wl) >= Nk - 1 && static_cast<long long>(w.wr) >= Nq - 1);
+  return w;
 }
 
-template <int D, bool CAUSAL, bool BF16>
+template <int D, bool BAND, bool BF16>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-               const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int BH,
-               int Nq, int Nk, float scale, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, BF16>;
+               const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int B,
+               int H, int Nq, int Nk, Window w, float scale, cudaStream_t stream) {
+  auto kern = fa::fa_fwd_kernel<D, BAND, BF16>;
   // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
   // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
   const int smem = fa::FwdLayout<D>::kBytes > 120 * 1024 ? fa::FwdLayout<D>::kBytes : 120 * 1024;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  const unsigned grid =
-      static_cast<unsigned>(BH) * static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk,
-                                                 scale * 1.4426950408889634074f);
+  const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) *
+                        static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
+  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
+                                                 w.wr, scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -131,7 +165,8 @@ struct BwdArgs {
   const CUtensorMap* k;
   const CUtensorMap* v;
   const CUtensorMap* dO_map;
-  const CUtensorMap* dq_map;
+  const CUtensorMap* dq_map;   // the fp32 dQ accumulator (reduce-add target)
+  const CUtensorMap* dq_out;   // dQ itself (deterministic mode: the dQ pass stores it)
   const void* O;
   const void* O_res;
   const void* dO;
@@ -139,36 +174,44 @@ struct BwdArgs {
   void* dQ;
   void* dK;
   void* dV;
-  int BH;
+  int B;
+  int H;
   int Nq;  // query rows (Q, O, dO, dQ, L, the workspace)
   int Nk;  // key rows (K, V, dK, dV)
+  int layout;
+  Window w;
+  bool det;  // deterministic: dQ by its own pass, no accumulator
   float scale;
   void* workspace;
   cudaStream_t stream;
 };
 
-enum { kStagePre = 1, kStageMain = 2, kStageDq = 4, kStageAll = 7 };
-
-// Workspace: D and Ls as [BH][n_pad] fp32 (n_pad = Nq rounded up to 128, so that every
-// query tile reads whole 512-byte rows), then the dQ accumulator [BH][Nq][d] fp32.
-template <int D, bool CAUSAL, bool BF16>
+// Workspace: D and Ls as [B*H][n_pad] fp32 (n_pad = Nq rounded up to 128, so that every
+// query tile reads whole 512-byte rows), then (not in deterministic mode) the dQ
+// accumulator [B*H][Nq][d] fp32.
+template <int D, bool BAND, bool BF16>
 int launch_bwd(const BwdArgs& a, int stages) {
-  const long rows = static_cast<long>(a.BH) * a.Nq;
+  const int BH = a.B * a.H;
+  const long rows = static_cast<long>(BH) * a.Nq;
   const int n_pad = (a.Nq + fa::kTile - 1) / fa::kTile * fa::kTile;
-  const long prows = static_cast<long>(a.BH) * n_pad;
+  const long prows = static_cast<long>(BH) * n_pad;
   float* Dv = static_cast<float*>(a.workspace);
   float* Ls = Dv + prows;
-  float* dq_acc = Ls + prows;
-  if (stages & kStagePre) {
+  float* dq_acc = a.det ? nullptr : Ls + prows;
+  const fa::Strides sq = strides_of(a.layout, a.H, a.Nq, D);
+  const fa::Strides sk = strides_of(a.layout, a.H, a.Nk, D);
+  const float scale_log2 = a.scale * 1.4426950408889634074f;
+  if (stages & FA_STAGE_PREPROCESS) {
     const long threads = prows * (D / 8);
     const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
     fa::fa_bwd_pre_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
         static_cast<const uint16_t*>(a.O), static_cast<const uint16_t*>(a.O_res),
-        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, a.Nq, n_pad, prows);
+        static_cast<const uint16_t*>(a.dO), a.L, Dv, Ls, dq_acc, a.Nq, n_pad, prows, a.H, sq);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  if (stages & kStageMain) {
-    auto kern = fa::fa_bwd_main_kernel<D, CAUSAL, BF16>;
+  if (stages & FA_STAGE_DKDV) {
+    auto kern = a.det ? fa::fa_bwd_main_kernel<D, BAND, BF16, false>
+                      : fa::fa_bwd_main_kernel<D, BAND, BF16, true>;
     const size_t need = fa::BwdLayout<D>::kNeeded;
     if (need > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
     const size_t smem = need + 1024 <= kMaxDynSmem ? need + 1024 : kMaxDynSmem;
@@ -177,37 +220,51 @@ int launch_bwd(const BwdArgs& a, int stages) {
       return FA_ERR_CUDA;
     // The kernel moves registers between warpgroups (setmaxnreg); its split adds up to
     // exactly 128 registers per thread at launch. Launched with fewer, the increase
-    // would wait for registers that never come back, so refuse instead.
+    // would wait for registers that never come back, so refuse instead (the build
+    // also fails for such a kernel).
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FA_ERR_CUDA;
     if (attr.numRegs != fa::kBwdLaunchRegs) return FA_ERR_UNSUPPORTED;
-    const unsigned grid =  // one CTA per key tile
-        static_cast<unsigned>(a.BH) * static_cast<unsigned>((a.Nk + fa::kTile - 1) / fa::kTile);
+    const unsigned grid = static_cast<unsigned>(BH) *  // one CTA per key tile
+                          static_cast<unsigned>((a.Nk + fa::kTile - 1) / fa::kTile);
     kern<<<grid, fa::kBwdThreads, smem, a.stream>>>(
         *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
-        static_cast<uint16_t*>(a.dV), a.Nq, a.Nk, a.scale, a.scale * 1.4426950408889634074f,
+        static_cast<uint16_t*>(a.dV), a.Nq, a.Nk, a.H, a.w.wl, a.w.wr, sk, a.scale, scale_log2,
         static_cast<uint32_t>(smem));
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
-  if (stages & kStageDq) {
+  if ((stages & FA_STAGE_DQ) && a.det) {
+    auto kern = fa::fa_bwd_dq_pass_kernel<D, BAND, BF16>;
+    const int smem = fa::DqLayout<D>::kBytes > 120 * 1024 ? fa::DqLayout<D>::kBytes : 120 * 1024;
+    if (static_cast<size_t>(smem) > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    const unsigned grid = static_cast<unsigned>(BH) *  // one CTA per query tile
+                          static_cast<unsigned>((a.Nq + fa::kTile - 1) / fa::kTile);
+    kern<<<grid, fa::kDqThreads, smem, a.stream>>>(*a.q, *a.k, *a.v, *a.dO_map, *a.dq_out, Ls,
+                                                   Dv, a.Nq, a.Nk, a.H, a.w.wl, a.w.wr, a.scale,
+                                                   scale_log2);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  } else if (stages & FA_STAGE_DQ) {
     const long n8 = rows * D / 8;
     const unsigned blocks = static_cast<unsigned>((n8 + 255) / 256);
     fa::fa_bwd_dq_kernel<D, BF16><<<blocks, 256, 0, a.stream>>>(
-        dq_acc, static_cast<uint16_t*>(a.dQ), a.scale, n8);
+        dq_acc, static_cast<uint16_t*>(a.dQ), a.scale, n8, a.Nq, a.H, sq);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   return FA_OK;
 }
 
-// Compile-time dispatch over (d, causal, dtype).
+// Compile-time dispatch over (d, band, dtype).
 template <template <int, bool, bool> class F, typename... Args>
-int dispatch(int d, int causal, int dtype, Args&&... args) {
+int dispatch(int d, bool band, int dtype, Args&&... args) {
   const bool bf = dtype == FA_BF16;
   if (d == 64) {
-    if (causal) return bf ? F<64, true, true>::run(args...) : F<64, true, false>::run(args...);
+    if (band) return bf ? F<64, true, true>::run(args...) : F<64, true, false>::run(args...);
     return bf ? F<64, false, true>::run(args...) : F<64, false, false>::run(args...);
   }
-  if (causal) return bf ? F<128, true, true>::run(args...) : F<128, true, false>::run(args...);
+  if (band) return bf ? F<128, true, true>::run(args...) : F<128, true, false>::run(args...);
   return bf ? F<128, false, true>::run(args...) : F<128, false, false>::run(args...);
 }
 
@@ -220,6 +277,147 @@ template <int D, bool C, bool B>
 struct BwdRun {
   template <typename... A>
   static int run(A&&... a) { return launch_bwd<D, C, B>(a...); }
+};
+
+size_t workspace_bytes_for(int B, int H, int Nq, int d, bool det) {
+  const size_t rows = static_cast<size_t>(B) * H * Nq;
+  if (rows == 0) return 0;
+  // D and Ls (fp32 per row, Nq padded to a multiple of 128 per head), then the fp32 dQ
+  // accumulator; its start is 1024-byte aligned because the padded row count is a
+  // multiple of 128. The deterministic mode forms dQ in its own pass and keeps no
+  // accumulator.
+  const size_t n_pad = (static_cast<size_t>(Nq) + 127) / 128 * 128;
+  const size_t stats = static_cast<size_t>(B) * H * n_pad * 4 * 2;
+  return det ? stats : stats + rows * static_cast<size_t>(d) * 4;
+}
+
+// The backward (all stages, or the ones in `stages`), checked like fa_bwd_ex. Pointers
+// a stage does not use may be NULL when only that stage runs.
+int bwd_checked(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
+                const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H,
+                int Nq, int Nk, int d, int layout, int window_left, int window_right,
+                int deterministic, float scale, int dtype, void* workspace,
+                size_t workspace_bytes, void* stream, int stages) {
+  bool empty;
+  int st = check_shape(B, H, Nq, Nk, d, layout, dtype, scale, &empty);
+  if (st != FA_OK) return st;
+  if (deterministic != 0 && deterministic != 1) return FA_ERR_INVALID;
+  if (stages <= 0 || stages > FA_STAGE_ALL) return FA_ERR_INVALID;
+  const bool det = deterministic != 0;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (empty) {
+    // no query rows: every key's gradient is an empty sum
+    if (!(stages & FA_STAGE_DKDV)) return FA_OK;
+    const size_t bytes = static_cast<size_t>(B) * H * Nk * d * 2;
+    if (bytes == 0) return FA_OK;
+    if (!ok_ptr(dK) || !ok_ptr(dV)) return FA_ERR_INVALID;
+    return cudaMemsetAsync(dK, 0, bytes, s) == cudaSuccess &&
+                   cudaMemsetAsync(dV, 0, bytes, s) == cudaSuccess
+               ? FA_OK
+               : FA_ERR_CUDA;
+  }
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID;
+  if (workspace_bytes < workspace_bytes_for(B, H, Nq, d, det)) return FA_ERR_INVALID;
+  if (!aligned16(O_res)) return FA_ERR_INVALID;
+  if ((stages & FA_STAGE_PREPROCESS) && (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L)))
+    return FA_ERR_INVALID;
+  if ((stages & FA_STAGE_DKDV) &&
+      (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO) || !ok_ptr(dK) || !ok_ptr(dV)))
+    return FA_ERR_INVALID;
+  if ((stages & FA_STAGE_DQ) && !ok_ptr(dQ)) return FA_ERR_INVALID;
+  if (det && (stages & FA_STAGE_DQ) &&
+      (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO)))  // the dQ pass reads them
+    return FA_ERR_INVALID;
+  const Window w = window_of(Nq, Nk, window_left, window_right);
+  const int BH = B * H;
+  const long prows = static_cast<long>(BH) * ((Nq + fa::kTile - 1) / fa::kTile * fa::kTile);
+  CUtensorMap tq, tk, tv, tdo, tdq, tdqo;
+  if ((stages & FA_STAGE_DKDV) || (det && (stages & FA_STAGE_DQ))) {
+    if (!make_tmap(&tq, Q, B, H, Nq, d, layout, dtype) ||
+        !make_tmap(&tk, K, B, H, Nk, d, layout, dtype) ||
+        !make_tmap(&tv, V, B, H, Nk, d, layout, dtype) ||
+        !make_tmap(&tdo, dO, B, H, Nq, d, layout, dtype))
+      return FA_ERR_CUDA;
+  }
+  // the accumulator's map (a deterministic run never touches it, so any valid base works)
+  const float* dq_acc = static_cast<const float*>(workspace) + (det ? 0 : 2 * prows);
+  if ((stages & FA_STAGE_DKDV) && !make_tmap_f32(&tdq, dq_acc, B, H, Nq, d)) return FA_ERR_CUDA;
+  if (det && (stages & FA_STAGE_DQ) && !make_tmap(&tdqo, dQ, B, H, Nq, d, layout, dtype))
+    return FA_ERR_CUDA;
+  BwdArgs a{&tq,  &tk, &tv, &tdo, &tdq,   &tdqo, O,   O_res, dO,    L,         dQ,
+            dK,   dV,  B,   H,    Nq,     Nk,    layout, w,  det,   scale,     workspace, s};
+  return dispatch<BwdRun>(d, w.band, dtype, a, stages);
+}
+
+// ------------------------------------------------------------------- decode
+// Key tiles that the decode rows (Nq <= 16, all in query tile 0) visit together.
+fa::TileRange decode_tiles(int Nq, int Nk, const Window& w) {
+  const int ntk = (Nk + fa::kTile - 1) / fa::kTile;
+  return w.band ? fa::kv_tiles_of_query_tile(0, fa::kTile, Nq, Nk, w.wl, w.wr)
+                : fa::TileRange{0, ntk};
+}
+
+// Splits per head: the count that minimises the estimated time, (waves of 148 CTAs,
+// one CTA per SM) x (tiles per split + a fixed cost of about two tiles per CTA). A
+// fixed SM count keeps the split -- and so the rounding of the merge -- the same on
+// every B200.
+int decode_splits(long BH, int ntiles) {
+  if (ntiles <= 1) return 1;
+  constexpr long kSms = 148;
+  int best = 1;
+  long best_cost = -1;
+  const int max_s = ntiles < 1024 ? ntiles : 1024;
+  for (int s = 1; s <= max_s; ++s) {
+    const int tps = (ntiles + s - 1) / s;
+    if ((ntiles + tps - 1) / tps != s) continue;  // every split gets at least one tile
+    const long waves = (BH * s + kSms - 1) / kSms;
+    const long cost = waves * (tps + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+size_t decode_workspace(long BH, int Nq, int d, int splits) {
+  return splits <= 1 ? 0 : static_cast<size_t>(BH) * splits * Nq * (static_cast<size_t>(d) + 1) * 4;
+}
+
+template <int D, int NQ, bool BAND, bool BF16>
+int launch_decode_nq(const CUtensorMap& k, const CUtensorMap& v, const void* Q,
+                     const fa::Strides& sq, void* O, float* L, float* opart, float* lpart, int B,
+                     int H, int Nq, int Nk, const Window& w, fa::TileRange tiles, int splits,
+                     float scale, cudaStream_t stream) {
+  auto kern = fa::fa_decode_kernel<D, NQ, BAND, BF16>;
+  const int smem = fa::DecLayout<D>::kBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  const long BH = static_cast<long>(B) * H;
+  const int tps = tiles.count > 0 ? (tiles.count + splits - 1) / splits : 0;
+  kern<<<static_cast<unsigned>(BH * splits), fa::dec_threads(NQ), smem, stream>>>(
+      k, v, static_cast<const uint16_t*>(Q), sq, static_cast<uint16_t*>(O), sq, L, opart, lpart,
+      Nq, Nk, H, w.wl, w.wr, tiles.first, tiles.count, tps, splits,
+      scale * 1.4426950408889634074f);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (splits > 1) {
+    const long rows = BH * Nq;
+    fa::fa_decode_merge_kernel<D, BF16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        opart, lpart, static_cast<uint16_t*>(O), sq, L, Nq, H, splits, rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+template <int D, bool BAND, bool BF16>
+struct DecodeRun {
+  template <typename... A>
+  static int run(int Nq, A&&... a) {
+    if (Nq <= 1) return launch_decode_nq<D, 1, BAND, BF16>(a...);
+    if (Nq <= 4) return launch_decode_nq<D, 4, BAND, BF16>(a...);
+    return launch_decode_nq<D, 16, BAND, BF16>(a...);
+  }
 };
 
 // ------------------------------------------------ backward without allocation
@@ -262,24 +460,31 @@ const char* fa_status_string(int status) {
   }
 }
 
+int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L,
+              int B, int H, int Nq, int Nk, int d, int layout, int window_left,
+              int window_right, float scale, int dtype, void* stream) {
+  bool empty;
+  int st = check_shape(B, H, Nq, Nk, d, layout, dtype, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(L) || !aligned16(O_res))
+    return FA_ERR_INVALID;
+  CUtensorMap tq, tk, tv, to, tr;
+  if (!make_tmap(&tq, Q, B, H, Nq, d, layout, dtype) ||
+      !make_tmap(&tk, K, B, H, Nk, d, layout, dtype) ||
+      !make_tmap(&tv, V, B, H, Nk, d, layout, dtype) ||
+      !make_tmap(&to, O, B, H, Nq, d, layout, dtype) ||
+      !make_tmap(&tr, O_res != nullptr ? O_res : O, B, H, Nq, d, layout, dtype))
+    return FA_ERR_CUDA;
+  const Window w = window_of(Nq, Nk, window_left, window_right);
+  return dispatch<FwdRun>(d, w.band, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
+                          Nk, w, scale, static_cast<cudaStream_t>(stream));
+}
+
 int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L,
               int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
               void* stream) {
-  bool empty;
-  int st = check_shape_qk(B, H, Nq, Nk, d, dtype, scale, &empty);
-  if (st != FA_OK || empty) return st;
-  if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L) ||
-      !aligned16(O_res))
-    return FA_ERR_INVALID;
-  const int BH = B * H;
-  CUtensorMap tq, tk, tv, to, tr;
-  if (!make_tmap(&tq, Q, BH, Nq, d, dtype) || !make_tmap(&tk, K, BH, Nk, d, dtype) ||
-      !make_tmap(&tv, V, BH, Nk, d, dtype) || !make_tmap(&to, O, BH, Nq, d, dtype) ||
-      !make_tmap(&tr, O_res != nullptr ? O_res : O, BH, Nq, d, dtype))
-    return FA_ERR_CUDA;
-  return dispatch<FwdRun>(d, causal, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, BH, Nq, Nk,
-                          scale, static_cast<cudaStream_t>(stream));
+  return fa_fwd_ex(Q, K, V, O, O_res, L, B, H, Nq, Nk, d, FA_LAYOUT_BHND, -1, causal ? 0 : -1,
+                   scale, dtype, stream);
 }
 
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L, int B,
@@ -287,76 +492,40 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, void* O_res, fl
   return fa_fwd_qk(Q, K, V, O, O_res, L, B, H, N, N, d, causal, scale, dtype, stream);
 }
 
+size_t fa_bwd_ex_workspace_size(int B, int H, int Nq, int Nk, int d, int deterministic) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return static_cast<size_t>(-1);
+  return workspace_bytes_for(B, H, Nq, d, deterministic != 0);
+}
+
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
-  if (B < 0 || H < 0 || N < 0 || d < 0) return static_cast<size_t>(-1);
-  const size_t rows = static_cast<size_t>(B) * H * N;
-  if (rows == 0) return 0;
-  // D and Ls (fp32 per row, N padded to a multiple of 128 per head), then the fp32 dQ
-  // accumulator; its start is 1024-byte aligned because the padded row count is a
-  // multiple of 128.
-  const size_t n_pad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  return static_cast<size_t>(B) * H * n_pad * 4 * 2 + rows * static_cast<size_t>(d) * 4;
+  return fa_bwd_ex_workspace_size(B, H, N, N, d, 0);
 }
 
-// Validation shared by fa_bwd and its stages; the pointers a stage does not use may
-// be NULL (checked by the caller).
-static int bwd_common_qk(int B, int H, int Nq, int Nk, int d, int dtype, float scale,
-                         void* workspace, size_t workspace_bytes, bool* empty) {
-  int st = check_shape_qk(B, H, Nq, Nk, d, dtype, scale, empty);
-  if (st != FA_OK || *empty) return st;
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID;
-  if (workspace_bytes < fa_bwd_workspace_size(B, H, Nq, d)) return FA_ERR_INVALID;
-  return FA_OK;
-}
-static int bwd_common(int B, int H, int N, int d, int dtype, float scale, void* workspace,
-                      size_t workspace_bytes, bool* empty) {
-  return bwd_common_qk(B, H, N, N, d, dtype, scale, workspace, workspace_bytes, empty);
+int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
+              const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq,
+              int Nk, int d, int layout, int window_left, int window_right, int deterministic,
+              float scale, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_checked(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, Nq, Nk, d, layout, window_left,
+                     window_right, deterministic, scale, dtype, workspace, workspace_bytes,
+                     stream, FA_STAGE_ALL);
 }
 
-static int bwd_run(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
-                   const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H,
-                   int Nq, int Nk, int d, int causal, float scale, int dtype, void* workspace,
-                   void* stream, int stages) {
-  const int BH = B * H;
-  const long prows = static_cast<long>(BH) * ((Nq + fa::kTile - 1) / fa::kTile * fa::kTile);
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  if (stages & kStageMain) {
-    const float* dq_acc = static_cast<const float*>(workspace) + 2 * prows;
-    if (!make_tmap(&tq, Q, BH, Nq, d, dtype) || !make_tmap(&tk, K, BH, Nk, d, dtype) ||
-        !make_tmap(&tv, V, BH, Nk, d, dtype) || !make_tmap(&tdo, dO, BH, Nq, d, dtype) ||
-        !make_tmap_f32(&tdq, dq_acc, BH, Nq, d))
-      return FA_ERR_CUDA;
-  }
-  BwdArgs a{&tq, &tk, &tv, &tdo, &tdq, O, O_res, dO, L, dQ, dK, dV, BH, Nq, Nk, scale, workspace,
-            static_cast<cudaStream_t>(stream)};
-  return dispatch<BwdRun>(d, causal, dtype, a, stages);
+int fa_bwd_ex_stage(int stages, const void* Q, const void* K, const void* V, const void* O,
+                    const void* O_res, const void* dO, const float* L, void* dQ, void* dK,
+                    void* dV, int B, int H, int Nq, int Nk, int d, int layout, int window_left,
+                    int window_right, int deterministic, float scale, int dtype, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  return bwd_checked(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, Nq, Nk, d, layout, window_left,
+                     window_right, deterministic, scale, dtype, workspace, workspace_bytes,
+                     stream, stages);
 }
-
-static bool ok_ptr(const void* p) { return p && aligned16(p); }
 
 int fa_bwd_qk(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
               const void* dO, const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, void* workspace,
               size_t workspace_bytes, void* stream) {
-  bool empty;
-  int st = bwd_common_qk(B, H, Nq, Nk, d, dtype, scale, workspace, workspace_bytes, &empty);
-  if (st != FA_OK) return st;
-  if (empty) {
-    // no query rows: every key's gradient is an empty sum
-    const size_t bytes = static_cast<size_t>(B) * H * Nk * d * 2;
-    if (bytes == 0) return FA_OK;
-    if (!ok_ptr(dK) || !ok_ptr(dV)) return FA_ERR_INVALID;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    return cudaMemsetAsync(dK, 0, bytes, s) == cudaSuccess &&
-                   cudaMemsetAsync(dV, 0, bytes, s) == cudaSuccess
-               ? FA_OK
-               : FA_ERR_CUDA;
-  }
-  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
-      !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
-    return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, Nq, Nk, d, causal, scale, dtype,
-                 workspace, stream, kStageAll);
+  return fa_bwd_ex(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, Nq, Nk, d, FA_LAYOUT_BHND, -1,
+                   causal ? 0 : -1, 0, scale, dtype, workspace, workspace_bytes, stream);
 }
 
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* O_res,
@@ -370,34 +539,86 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
 int fa_bwd_preprocess(const void* O, const void* O_res, const void* dO, const float* L, int B,
                       int H, int N, int d, int dtype, void* workspace, size_t workspace_bytes,
                       void* stream) {
-  bool empty;
-  int st = bwd_common(B, H, N, d, dtype, 1.f, workspace, workspace_bytes, &empty);
-  if (st != FA_OK || empty) return st;
-  if (!ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) || !aligned16(O_res)) return FA_ERR_INVALID;
-  return bwd_run(nullptr, nullptr, nullptr, O, O_res, dO, L, nullptr, nullptr, nullptr, B, H, N,
-                 N, d, 0, 1.f, dtype, workspace, stream, kStagePre);
+  return bwd_checked(nullptr, nullptr, nullptr, O, O_res, dO, L, nullptr, nullptr, nullptr, B, H,
+                     N, N, d, FA_LAYOUT_BHND, -1, -1, 0, 1.f, dtype, workspace, workspace_bytes,
+                     stream, FA_STAGE_PREPROCESS);
 }
 
 int fa_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
                 int B, int H, int N, int d, int causal, float scale, int dtype, void* workspace,
                 size_t workspace_bytes, void* stream) {
-  bool empty;
-  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
-  if (st != FA_OK || empty) return st;
-  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(dO) || !ok_ptr(dK) || !ok_ptr(dV))
-    return FA_ERR_INVALID;
-  return bwd_run(Q, K, V, nullptr, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, N, d, causal,
-                 scale, dtype, workspace, stream, kStageMain);
+  return bwd_checked(Q, K, V, nullptr, nullptr, dO, nullptr, nullptr, dK, dV, B, H, N, N, d,
+                     FA_LAYOUT_BHND, -1, causal ? 0 : -1, 0, scale, dtype, workspace,
+                     workspace_bytes, stream, FA_STAGE_DKDV);
 }
 
 int fa_bwd_dq_convert(void* dQ, int B, int H, int N, int d, float scale, int dtype,
                       void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_checked(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
+                     nullptr, B, H, N, N, d, FA_LAYOUT_BHND, -1, -1, 0, scale, dtype, workspace,
+                     workspace_bytes, stream, FA_STAGE_DQ);
+}
+
+int fa_tile_range(int query_side, int tile, int Nq, int Nk, int window_left, int window_right,
+                  int* first, int* count) {
+  if (!first || !count || Nq <= 0 || Nk <= 0 || tile < 0 ||
+      static_cast<long long>(Nq) + Nk > kMaxRowsPerHead)
+    return FA_ERR_INVALID;
+  const Window w = window_of(Nq, Nk, window_left, window_right);
+  const int ntq = (Nq + fa::kTile - 1) / fa::kTile;
+  const int ntk = (Nk + fa::kTile - 1) / fa::kTile;
+  fa::TileRange r;
+  if (query_side) {
+    if (tile >= ntq) return FA_ERR_INVALID;
+    r = w.band ? fa::kv_tiles_of_query_tile(tile, fa::kTile, Nq, Nk, w.wl, w.wr)
+               : fa::TileRange{0, ntk};
+  } else {
+    if (tile >= ntk) return FA_ERR_INVALID;
+    r = w.band ? fa::query_tiles_of_kv_tile(tile, fa::kTile, Nq, Nk, w.wl, w.wr)
+               : fa::TileRange{0, ntq};
+  }
+  *first = r.first;
+  *count = r.count;
+  return FA_OK;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int window_left,
+                                int window_right) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return static_cast<size_t>(-1);
+  if (static_cast<long long>(B) * H * Nq == 0 || Nk == 0 || Nq > fa::kDecMaxQ ||
+      static_cast<long long>(Nq) + Nk > kMaxRowsPerHead)
+    return 0;
+  const Window w = window_of(Nq, Nk, window_left, window_right);
+  const long BH = static_cast<long>(B) * H;
+  return decode_workspace(BH, Nq, d, decode_splits(BH, decode_tiles(Nq, Nk, w).count));
+}
+
+int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
+              int Nq, int Nk, int d, int layout, int window_left, int window_right, float scale,
+              int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   bool empty;
-  int st = bwd_common(B, H, N, d, dtype, scale, workspace, workspace_bytes, &empty);
+  int st = check_shape(B, H, Nq, Nk, d, layout, dtype, scale, &empty);
   if (st != FA_OK || empty) return st;
-  if (!ok_ptr(dQ)) return FA_ERR_INVALID;
-  return bwd_run(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dQ, nullptr,
-                 nullptr, B, H, N, N, d, 0, scale, dtype, workspace, stream, kStageDq);
+  if (Nq > fa::kDecMaxQ) return FA_ERR_UNSUPPORTED;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(L)) return FA_ERR_INVALID;
+  const Window w = window_of(Nq, Nk, window_left, window_right);
+  const long BH = static_cast<long>(B) * H;
+  const fa::TileRange tiles = decode_tiles(Nq, Nk, w);
+  const int splits = decode_splits(BH, tiles.count);
+  const size_t need = decode_workspace(BH, Nq, d, splits);
+  if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+                   workspace_bytes < need))
+    return FA_ERR_INVALID;
+  if (BH * splits >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  CUtensorMap tk, tv;
+  if (!make_tmap(&tk, K, B, H, Nk, d, layout, dtype) ||
+      !make_tmap(&tv, V, B, H, Nk, d, layout, dtype))
+    return FA_ERR_CUDA;
+  float* opart = static_cast<float*>(workspace);
+  float* lpart = splits > 1 ? opart + BH * splits * Nq * d : nullptr;
+  const fa::Strides sq = strides_of(layout, H, Nq, d);
+  return dispatch<DecodeRun>(d, w.band, dtype, Nq, tk, tv, Q, sq, O, L, opart, lpart, B, H, Nq,
+                             Nk, w, tiles, splits, scale, static_cast<cudaStream_t>(stream));
 }
 
 int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
@@ -410,15 +631,15 @@ int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
   if (need == static_cast<size_t>(-1)) return FA_ERR_INVALID;
   if (need > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
   bool empty;
-  int st = check_shape(B, H, N, d, dtype, scale, &empty);
+  int st = check_shape(B, H, N, N, d, FA_LAYOUT_BHND, dtype, scale, &empty);
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(dO) || !ok_ptr(L) ||
       !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !aligned16(O_res))
     return FA_ERR_INVALID;
   void* scratch = noalloc_scratch_address(&st);
   if (st != FA_OK) return st;
-  return bwd_run(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, N, d, causal, scale, dtype,
-                 scratch, stream, kStageAll);
+  return fa_bwd(Q, K, V, O, O_res, dO, L, dQ, dK, dV, B, H, N, d, causal, scale, dtype, scratch,
+                kNoAllocScratchBytes, stream);
 }
 
 int fa_selftest_wait_timeout(long long limit_cycles, void* stream) {

@@ -1,0 +1,61 @@
+// fa_band.cuh -- which key/value tiles a query tile visits, and the reverse, for the
+// masks the kernels support (host and device code share these).
+//
+// Every mask is a key window around the bottom-right diagonal: with off = Nk - Nq,
+// query q sees key k iff q + off - wl <= k <= q + off + wr (and 0 <= k < Nk). The
+// unmasked case is wl = wr = kUnbounded; the causal mask is wl = kUnbounded, wr = 0;
+// a sliding window bounds either side (josueisai.com "flash-attention", section "Que
+// ganas y que no", names window attention as the combination for very long
+// sequences). Tiles outside the band are never loaded or multiplied; tiles across
+// an edge of the band are masked element by element.
+#pragma once
+
+namespace fa {
+
+// An edge at least this far from the diagonal bounds nothing (the host clamps every
+// window to this, and keeps Nq + Nk below it, so no sum here overflows 32 bits).
+constexpr int kUnbounded = 1 << 30;
+
+// Element strides of a 16-bit [B][H][N][d] or [B][N][H][d] tensor: element (b, h, n, t)
+// sits at b * sb + h * sh + n * sn + t.
+struct Strides {
+  long sb, sh, sn;
+};
+
+struct TileRange {
+  int first;  // first tile index
+  int count;  // number of consecutive tiles (0: none)
+};
+
+// Key/value tiles (of `tile` keys) that query tile t (rows t*tile .. t*tile+tile-1,
+// the last possibly past Nq) has to visit: the union of its rows' windows.
+__host__ __device__ inline TileRange kv_tiles_of_query_tile(int t, int tile, int Nq, int Nk,
+                                                            int wl, int wr) {
+  const int off = Nk - Nq;
+  const int q0 = t * tile;
+  const int q1 = t * tile + tile - 1 < Nq - 1 ? t * tile + tile - 1 : Nq - 1;  // last real row
+  const int lo = q0 + off - wl;  // smallest key any row of the tile sees
+  const int hi = q1 + off + wr;  // largest
+  const int klo = lo < 0 ? 0 : lo;
+  const int khi = hi > Nk - 1 ? Nk - 1 : hi;
+  if (klo > khi) return {0, 0};
+  return {klo / tile, khi / tile - klo / tile + 1};
+}
+
+// Query tiles whose rows see at least one key of key tile j (rows of the last query
+// tile past Nq included: they are padding and see what the window gives them).
+__host__ __device__ inline TileRange query_tiles_of_kv_tile(int j, int tile, int Nq, int Nk,
+                                                            int wl, int wr) {
+  const int off = Nk - Nq;
+  const int k0 = j * tile;
+  const int k1 = j * tile + tile - 1 < Nk - 1 ? j * tile + tile - 1 : Nk - 1;
+  const int lo = k0 - off - wr;  // smallest query that sees key k0 .. k1
+  const int hi = k1 - off + wl;  // largest
+  const int ntq = (Nq + tile - 1) / tile;
+  const int qlo = lo < 0 ? 0 : lo;
+  const int qhi = hi > ntq * tile - 1 ? ntq * tile - 1 : hi;
+  if (qlo > qhi) return {0, 0};
+  return {qlo / tile, qhi / tile - qlo / tile + 1};
+}
+
+}  // namespace fa

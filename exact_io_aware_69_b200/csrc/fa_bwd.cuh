@@ -44,6 +44,7 @@
 //   warps 14-15 idle (they complete warpgroup 3, which runs on 56 registers).
 #pragma once
 
+#include "fa_band.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -115,7 +116,8 @@ __global__ void __launch_bounds__(256)
     fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ O_res,
                       const uint16_t* __restrict__ dO, const float* __restrict__ L,
                       float* __restrict__ Dv, float* __restrict__ Ls,
-                      float* __restrict__ dq_acc, int N, int n_pad, long padded_rows) {
+                      float* __restrict__ dq_acc, int N, int n_pad, long padded_rows, int H,
+                      Strides st) {
   constexpr int kTpr = D / 8;  // threads per row
   const long gid = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long prow = gid / kTpr;  // row in the padded layout
@@ -123,12 +125,14 @@ __global__ void __launch_bounds__(256)
   const long bh = prow / n_pad;
   const int n = static_cast<int>(prow - bh * n_pad);
   const bool real = prow < padded_rows && n < N;
-  const long row = bh * N + n;  // row in the [B*H*N, D] tensors (when real)
+  const long row = bh * N + n;  // row of L and of the dQ accumulator ([B][H][N] order)
+  const int bhi = static_cast<int>(bh);  // < 2^31 (checked on the host)
+  const long el = (bhi / H) * st.sb + (bhi % H) * st.sh + n * st.sn + part * 8;  // O, dO
   float acc = 0.f;
   if (real) {
-    const uint4 o = *reinterpret_cast<const uint4*>(O + row * D + part * 8);
-    const uint4 g = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
-    const uint4 res = O_res != nullptr ? *reinterpret_cast<const uint4*>(O_res + row * D + part * 8)
+    const uint4 o = *reinterpret_cast<const uint4*>(O + el);
+    const uint4 g = *reinterpret_cast<const uint4*>(dO + el);
+    const uint4 res = O_res != nullptr ? *reinterpret_cast<const uint4*>(O_res + el)
                                        : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t* ow = reinterpret_cast<const uint32_t*>(&o);
     const uint32_t* rw = reinterpret_cast<const uint32_t*>(&res);
@@ -142,9 +146,11 @@ __global__ void __launch_bounds__(256)
       acc = fmaf(o0 + r0, g0, acc);
       acc = fmaf(o1 + r1, g1, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (dq_acc != nullptr) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + row * D + part * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 #pragma unroll
   for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
@@ -156,10 +162,11 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------------ dQ convert
+// dQ = dtype(scale * dQacc); the accumulator is [B*H][N][D] fp32, dQ has strides `st`.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256)
     fa_bwd_dq_kernel(const float* __restrict__ dq_acc, uint16_t* __restrict__ dQ, float scale,
-                     long n8) {
+                     long n8, int N, int H, Strides st) {
   const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const float4 a = reinterpret_cast<const float4*>(dq_acc)[2 * i];
@@ -169,11 +176,19 @@ __global__ void __launch_bounds__(256)
   out.y = pack2<BF16>(a.z * scale, a.w * scale);
   out.z = pack2<BF16>(b.x * scale, b.y * scale);
   out.w = pack2<BF16>(b.z * scale, b.w * scale);
-  reinterpret_cast<uint4*>(dQ)[i] = out;
+  const long row = i / (D / 8);
+  const int part = static_cast<int>(i - row * (D / 8));
+  const int bh = static_cast<int>(row / N);  // < 2^31 (checked on the host)
+  const long n = row - static_cast<long>(bh) * N;
+  *reinterpret_cast<uint4*>(dQ + (bh / H) * st.sb + (bh % H) * st.sh + n * st.sn + part * 8) =
+      out;
 }
 
 // --------------------------------------------------------------- main dK/dV
-template <int D, bool CAUSAL, bool BF16>
+// BAND as in the forward: false = every key visible, true = the key window [wl, wr]
+// (causal: wl = kUnbounded, wr = 0). dK and dV are written with element strides `kv`.
+// DQ = false leaves dQ to the separate pass of fa_bwd_dq.cuh: no dQ MMA, no drain.
+template <int D, bool BAND, bool BF16, bool DQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -182,7 +197,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ Ls,
                        const float* __restrict__ Dv, float* __restrict__ dq_acc,
                        uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int Nq, int Nk,
-                       float scale, float scale_log2, uint32_t smem_alloc) {
+                       int H, int wl, int wr, Strides kv, float scale, float scale_log2,
+                       uint32_t smem_alloc) {
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -201,20 +217,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head
   const int ntk = (Nk + kTile - 1) / kTile;  // key tiles per head (one CTA each)
   const int bh = blockIdx.x / ntk;
+  const int hh = bh % H;  // head
+  const int bb = bh / H;  // batch
   const int j = blockIdx.x - bh * ntk;  // key tile (j = 0 has the most causal work)
-  // Rows past Nq / Nk arrive as zeros through the 3-D tensor maps. Padded queries, and
+  // Rows past Nq / Nk arrive as zeros through the tensor maps. Padded queries, and
   // queries that see no key, have Ls = -inf, so their P is 0. Padded keys of the last
   // key tile need no mask: their dK and dV rows are not stored, and their dS meets
   // zero rows of K in dQ = dS K. Ls and Dv are laid out per head with ntq * 128 rows.
-  // Causal masking is bottom-right aligned (query q sees keys k <= q + off): the first
-  // query tile whose last row sees key j * 128 is i_begin; the last query sees every
-  // key, so niter >= 1.
+  // The query tiles walked are those with a row that sees a key of this tile (under
+  // the causal mask there is at least one, because the last query sees every key; a
+  // sliding window may leave a key tile unseen, and its dK, dV are then zero).
+  const TileRange qr = BAND ? query_tiles_of_kv_tile(j, kTile, Nq, Nk, wl, wr)
+                            : TileRange{0, ntq};
+  const int i_begin = qr.first;
+  const int niter = qr.count;
   const int off = Nk - Nq;
-  const int first_q = j * kTile - (kTile - 1) - off;  // i_begin = ceil(first_q / 128)
-  const int i_begin =
-      !CAUSAL || first_q <= 0 ? 0 : (first_q + kTile - 1) / kTile;
-  const int niter = ntq - i_begin;
-  const long head_row = static_cast<long>(bh) * Nk;  // this key tile's head, in K rows
 
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kAbort);
@@ -251,7 +268,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kBwdProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     setmaxnreg_dec<kBwdSmallRegs>();  // each role of warpgroup 3 gives registers back
-    if (lane == 0) {
+    if (lane == 0 && niter > 0) {
       tma_prefetch(&tmQ);
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
@@ -260,9 +277,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
       mbar_expect_tx(bar(kBbKVFull), 2 * Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sbase + Lay::kK + c * Lay::kChunkBytes, &tmK, c * 64, j * kTile, bh,
+        tma_load_4d(sbase + Lay::kK + c * Lay::kChunkBytes, &tmK, c * 64, j * kTile, hh, bb,
                     bar(kBbKVFull));
-        tma_load_3d(sbase + Lay::kV + c * Lay::kChunkBytes, &tmV, c * 64, j * kTile, bh,
+        tma_load_4d(sbase + Lay::kV + c * Lay::kChunkBytes, &tmV, c * 64, j * kTile, hh, bb,
                     bar(kBbKVFull));
       }
       for (int it = 0; it < niter; ++it) {
@@ -274,8 +291,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t full = bar(kBbQFull + st);
         mbar_expect_tx(full, Lay::kTileBytes + 2 * 512);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
-                      qtile, bh, full);
+          tma_load_4d(sbase + Lay::kQ + st * Lay::kTileBytes + c * Lay::kChunkBytes, &tmQ, c * 64,
+                      qtile, hh, bb, full);
         bulk_load(sbase + Lay::kL + st * 512, Ls + head_pad + qtile, 512, full);
         bulk_load(sbase + Lay::kDv + st * 512, Dv + head_pad + qtile, 512, full);
         if (it >= 1 &&
@@ -283,7 +300,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         mbar_expect_tx(bar(kBbDOFull), Lay::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sbase + Lay::kDO + c * Lay::kChunkBytes, &tmDO, c * 64, qtile, bh,
+          tma_load_4d(sbase + Lay::kDO + c * Lay::kChunkBytes, &tmDO, c * 64, qtile, hh, bb,
                       bar(kBbDOFull));
         FA_TRACE_EVENT(it, 0);
       }
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // current one, and dK/dQ of the current tile while they exponentiate the next.
     // G1(i+1) overwrites the S^T/P^T columns only after G3(i), which reads P^T, has
     // been issued (MMAs from one thread execute in issue order).
-    if (lane == 0) {
+    if (lane == 0 && niter > 0) {
       constexpr uint32_t id_sq = idesc_f16_f32(kTile, kTile, BF16, false, false);  // S^T, dP^T
       constexpr uint32_t id_acc = idesc_f16_f32(kTile, D, BF16, false, true);      // dV, dK
       constexpr uint32_t id_dq = idesc_f16_f32(kTile, D, BF16, true, true);        // dQ
@@ -319,8 +336,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t dq = sdesc_sw128(sbase + Lay::kQ + st * Lay::kTileBytes, 16, 1024);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tS, sdesc_step(dk_k, off), sdesc_step(dq, off), id_sq,
+          const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tS, sdesc_step(dk_k, koff), sdesc_step(dq, koff), id_sq,
                  k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbSFull));
@@ -332,8 +349,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDP, sdesc_step(dv_k, off), sdesc_step(ddo_k, off), id_sq,
+          const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tDP, sdesc_step(dv_k, koff), sdesc_step(ddo_k, koff), id_sq,
                  k > 0 ? 1u : 0u);
         }
         mma_commit(bar(kBbDPFull));
@@ -359,29 +376,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // G4, G5 once dS_i is in shared memory
         if (!mbar_wait(bar(kBbDSReady), ph, abort_flag)) break;
         FA_TRACE_EVENT(it, 1);
-        if (D != 128 && it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
+        if (DQ && D != 128 && it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
         tc_fence_after();
         // dK += dS^T Q_i
         const uint64_t dq_mn = sdesc_sw128(sq, Lay::kChunkBytes, 1024);
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
-          const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDK, sdesc_step(dds_k, off), sdesc_step(dq_mn, k * 2048), id_acc,
+          const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+          mma_ss(tmem + Lay::tDK, sdesc_step(dds_k, koff), sdesc_step(dq_mn, k * 2048), id_acc,
                  (it > 0 || k > 0) ? 1u : 0u);
         }
-        // dQ_i = dS K_j   (dS read M-major from the same shared tile)
+        if constexpr (DQ) {
+          // dQ_i = dS K_j   (dS read M-major from the same shared tile)
 #pragma unroll
-        for (int k = 0; k < kTile / 16; ++k)
-          mma_ss(tmem + Lay::tDQ, sdesc_step(dds_mn, k * 2048), sdesc_step(dk_mn, k * 2048),
-                 id_dq, k > 0 ? 1u : 0u);
+          for (int k = 0; k < kTile / 16; ++k)
+            mma_ss(tmem + Lay::tDQ, sdesc_step(dds_mn, k * 2048), sdesc_step(dk_mn, k * 2048),
+                   id_dq, k > 0 ? 1u : 0u);
+        }
         mma_commit(bar(kBbQEmpty + st));
         mma_commit(bar(kBbDSFree));
-        mma_commit(bar(kBbDQFull));
+        if constexpr (DQ) mma_commit(bar(kBbDQFull));
         FA_TRACE_EVENT(it, 6);
         if (it + 1 < niter) {
           // G2 of the next tile. At d = 128 its columns hold dQ_i until the drain has
           // copied it out.
-          if (D == 128 && !mbar_wait(bar(kBbDQEmpty), ph, abort_flag)) break;
+          if (DQ && D == 128 && !mbar_wait(bar(kBbDQEmpty), ph, abort_flag)) break;
           if (!issue_dp(it + 1)) break;
         }
       }
@@ -395,25 +414,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint8_t* sds_row = smem + Lay::kDS + half * Lay::kChunkBytes + r * 128;
     const int sw = r & 7;
+    // The two warps of a pair meet at one named barrier per query tile and leave the
+    // loop together: a failed wait is carried to the next meeting, where bar.red.and
+    // makes both warps see it, so that neither is ever left waiting there alone.
     bool ok = true;
-    for (int it = 0; it < niter && ok; ++it) {
+    for (int it = 0; it < niter; ++it) {
       const int st = it & 1;
       const uint32_t ph = static_cast<uint32_t>(it & 1);
-      // causal: query column qc is masked for key row r when qc < r - dl
+      // band: query column qc of tile i sees key row r when r - dl - wr <= qc <= r - dl + wl
       const int dl = (i_begin + it) * kTile + off - j * kTile;
-      const bool diag = CAUSAL && dl < kTile - 1;
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) &&
-                          mbar_wait(bar(kBbSFull), ph, abort_flag));
-      if (!ok) break;
-      if (threadIdx.x == 0) FA_TRACE_EVENT(it, 7);
-      tc_fence_after();
+      const bool lo_edge = BAND && dl + wr < kTile - 1;     // some columns below the band
+      const bool hi_edge = BAND && dl - wl > -(kTile - 1);  // some columns above it
+      const bool got = __all_sync(
+          0xffffffffu,
+          ok && mbar_wait(bar(kBbQFull + st), static_cast<uint32_t>(it >> 1) & 1, abort_flag) &&
+              mbar_wait(bar(kBbSFull), ph, abort_flag));
+      if (got && threadIdx.x == 0) FA_TRACE_EVENT(it, 7);
       const float* sL = reinterpret_cast<const float*>(smem + Lay::kL + st * 512) + half * 64;
       const float* sD = reinterpret_cast<const float*>(smem + Lay::kDv + st * 512) + half * 64;
       // Both halves load their S^T columns before either writes P^T: the packed P^T
       // of the upper half (columns 32-63) lands on S^T columns of the lower half.
       float p[64];
-      {
+      if (got) {
+        tc_fence_after();
         uint32_t sr[64];
         tmem_ld32(lane_base + Lay::tS + half * 64, sr);
         tmem_ld32(lane_base + Lay::tS + half * 64 + 32, sr + 32);
@@ -423,7 +446,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int q = 0; q < 64; ++q) p[q] = __uint_as_float(sr[q]);
       }
-      named_bar_sync(1 + quarter, 64);
+      ok = named_bar_and(1 + quarter, 64, got);
+      if (!ok) break;
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 8);
       const uint64_t c2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll
@@ -441,10 +465,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           p[q + 1] = ex2_approx(x1);
           p[q + 2] = ex2_approx(x2);
           p[q + 3] = ex2_approx(x3);
-          if (diag) {
+          if (lo_edge || hi_edge) {
+            // this half's first and last visible column
+            const int qmin = (lo_edge ? r - dl - wr : 0) - half * 64;
+            const int qmax = (hi_edge ? r - dl + wl : kTile - 1) - half * 64;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              if (half * 64 + q + e < r - dl) p[q + e] = 0.f;
+              if (q + e < qmin || q + e > qmax) p[q + e] = 0.f;
           }
         }
 #pragma unroll
@@ -457,7 +484,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 9);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(kBbDPFull), ph, abort_flag) &&
                                        (it == 0 || mbar_wait(bar(kBbDSFree), ph ^ 1u, abort_flag)));
-      if (!ok) break;
+      if (!ok) continue;  // the pair agrees at the next meeting (or after the loop)
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 10);
       tc_fence_after();
 #pragma unroll
@@ -495,22 +522,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(bar(kBbDSReady));  // dS^T is in shared memory: dK and dQ may go
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 11);
     }
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(bar(kBbDone), 0, abort_flag));
+    // A key tile that no query sees (possible under a sliding window) ran no MMA: its
+    // dK and dV rows are zero.
+    const bool seen = niter > 0;
+    ok = __all_sync(0xffffffffu, ok && (!seen || mbar_wait(bar(kBbDone), 0, abort_flag)));
     if (ok) {
-      tc_fence_after();
-      const long grow = head_row + static_cast<long>(j) * kTile + r;
-      const bool live_row = j * kTile + r < Nk;  // padded keys of the last tile are not stored
+      if (seen) tc_fence_after();
+      const int key = j * kTile + r;
+      const bool live_row = key < Nk;  // padded keys of the last tile are not stored
+      const long el = bb * kv.sb + hh * kv.sh + static_cast<long>(key) * kv.sn + half * (D / 2);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t col = (which == 0 ? Lay::tDV : Lay::tDK) + half * (D / 2);
         const float mul = which == 0 ? 1.f : scale;
-        uint16_t* dst_row = (which == 0 ? dV : dK) + grow * D + half * (D / 2);
+        uint16_t* dst_row = (which == 0 ? dV : dK) + el;
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
           uint32_t v[32];
-          tmem_ld32(lane_base + col + c * 32, v);
-          tmem_wait_ld();
-          reg_fence32(v);
+          if (seen) {
+            tmem_ld32(lane_base + col + c * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
           uint4 pk[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
@@ -539,7 +575,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t stage = sbase + Lay::kStage;
     uint8_t* stage_row = smem + Lay::kStage + qr * 128;
     const int sw = qr & 7;
-    for (int it = 0; it < niter; ++it) {
+    for (int it = 0; it < (DQ ? niter : 0); ++it) {
       // Each warp frees its TMEM lanes as soon as dQ_i is there (the next dP^T MMA
       // waits for that); the four warps agree before touching the shared staging
       // buffer, so that all of them meet every named barrier below.
@@ -578,7 +614,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (leader) {
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            tma_reduce_add_3d(&tmDQ, stage + h * Lay::kChunkBytes, 32 * (2 * rnd + h), qtile, bh);
+            tma_reduce_add_4d(&tmDQ, stage + h * Lay::kChunkBytes, 32 * (2 * rnd + h), qtile, hh,
+                              bb);
           bulk_commit();
         }
       }

@@ -45,6 +45,7 @@
 // is a small difference that this error swamps.
 #pragma once
 
+#include "fa_band.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -88,12 +89,17 @@ enum : int {
 };
 static_assert(kFwdNumBars <= 20, "barrier area");
 
-template <int D, bool CAUSAL, bool BF16>
+// BAND = false: every key is visible (no mask but the end of a ragged last key tile);
+// BAND = true: the key window [wl, wr] around the bottom-right diagonal (fa_band.cuh),
+// the causal mask being wl = kUnbounded, wr = 0. Tensors are seen through 4-D tensor
+// maps (column, row, head, batch); L is [B][H][Nq].
+template <int D, bool BAND, bool BF16>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmOres, bool has_res,
-                  float* __restrict__ Lse, int Nq, int Nk, float scale_log2) {
+                  float* __restrict__ Lse, int Nq, int Nk, int H, int wl, int wr,
+                  float scale_log2) {
   using Lay = FwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -107,17 +113,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head (one CTA each)
   const int ntk = (Nk + kTile - 1) / kTile;  // key / value tiles per head
   const int bh = blockIdx.x / ntq;
+  const int hh = bh % H;  // head
+  const int bb = bh / H;  // batch
   const int tr = blockIdx.x - bh * ntq;
-  const int t = CAUSAL ? (ntq - 1 - tr) : tr;  // heaviest causal tiles first
-  // Causal masking is bottom-right aligned: query q sees keys k <= q + off. The tile's
-  // last row sees keys up to kmax; tiles past it are never loaded. With Nq > Nk the
-  // first Nq - Nk queries see no key (O = 0, L = -inf); a tile of only such rows has
-  // nkv = 0.
+  const int t = BAND ? (ntq - 1 - tr) : tr;  // causal: heaviest tiles first
+  // The key/value tiles this query tile visits: all of them, or the band's. With
+  // Nq > Nk under the causal mask the first Nq - Nk queries see no key (O = 0,
+  // L = -inf); a tile of only such rows visits none.
+  const TileRange kv = BAND ? kv_tiles_of_query_tile(t, kTile, Nq, Nk, wl, wr)
+                            : TileRange{0, ntk};
+  const int j0 = kv.first;
+  const int nkv = kv.count;
   const int off = Nk - Nq;
-  const int kmax = t * kTile + kTile - 1 + off;
-  const int nkv = !CAUSAL ? ntk : (kmax < 0 ? 0 : min(ntk, kmax / kTile + 1));
-  // Rows and keys of a last tile past Nq / Nk come in as zeros from the 3-D tensor
-  // maps; the keys are masked below, the rows are not stored.
+  // Rows and keys of a last tile past Nq / Nk come in as zeros from the tensor maps;
+  // the keys are masked below, the rows are not stored.
   const int last_keys = Nk - (ntk - 1) * kTile;  // valid keys in the last KV tile
 
   auto bar = [&](int i) -> uint32_t { return sbase + Lay::kBar + 8u * i; };
@@ -160,9 +169,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch(&tmV);
       mbar_expect_tx(bar(kBarQFull), Lay::kTileBytes);
       for (int c = 0; c < D / 64; ++c)
-        tma_load_3d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, t * kTile, bh,
+        tma_load_4d(sbase + Lay::kQ + c * Lay::kChunkBytes, &tmQ, c * 64, t * kTile, hh, bb,
                     bar(kBarQFull));
-      // step s loads K_s and V_{s-1}
+      // step s loads K and V of the visited tiles s and s - 1
       for (int step = 0; step <= nkv; ++step) {
         if (step < nkv) {
           const int ks = step % kFwdKStages;
@@ -173,7 +182,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t sk = sbase + Lay::kK + ks * Lay::kTileBytes;
           mbar_expect_tx(bar(kBarKFull + ks), Lay::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sk + c * Lay::kChunkBytes, &tmK, c * 64, step * kTile, bh,
+            tma_load_4d(sk + c * Lay::kChunkBytes, &tmK, c * 64, (j0 + step) * kTile, hh, bb,
                         bar(kBarKFull + ks));
           FA_TRACE_EVENT(step, 8);
         }
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t sv = sbase + Lay::kV + vs * Lay::kTileBytes;
           mbar_expect_tx(bar(kBarVFull + vs), Lay::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sv + c * Lay::kChunkBytes, &tmV, c * 64, j * kTile, bh,
+            tma_load_4d(sv + c * Lay::kChunkBytes, &tmV, c * 64, (j0 + j) * kTile, hh, bb,
                         bar(kBarVFull + vs));
           FA_TRACE_EVENT(j, 9);
         }
@@ -209,8 +218,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t d_s = tmem + (j & 1) * 128;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint32_t off = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-            mma_ss(d_s, sdesc_advance(dq, off), sdesc_advance(dk, off), idesc_s, k > 0 ? 1u : 0u);
+            const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+            mma_ss(d_s, sdesc_advance(dq, koff), sdesc_advance(dk, koff), idesc_s,
+                   k > 0 ? 1u : 0u);
           }
           mma_commit(bar(kBarKEmpty + ks));
           mma_commit(bar(kBarSFull + (j & 1)));
@@ -272,17 +282,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         reg_fence32(sr + 32);
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sr[c]);
-        // causal: key column c is masked for row r when c > r + delta (the tiles
-        // along the diagonal band); last tile: keys >= Nk
-        const int delta = t * kTile + off - j * kTile;
-        const bool cmask = CAUSAL && delta < kTile - 1;
-        const bool kmask = j == ntk - 1 && last_keys < kTile;
-        if (cmask || kmask) {
-          int lim = kmask ? last_keys - 1 : kTile - 1;
-          if (cmask) lim = min(lim, r + delta);
-          lim -= half * 64;
+        // band: key column c of the tile is visible to row r when
+        // r + delta - wl <= c <= r + delta + wr; last tile: keys >= Nk are masked
+        const int jt = j0 + j;  // the key tile itself
+        const int delta = t * kTile + off - jt * kTile;
+        const bool hmask = BAND && delta + wr < kTile - 1;  // upper edge crosses the tile
+        const bool lmask = BAND && delta - wl > -(kTile - 1);  // lower edge crosses it
+        const bool kmask = jt == ntk - 1 && last_keys < kTile;
+        if (hmask || lmask || kmask) {
+          int hi = kmask ? last_keys - 1 : kTile - 1;
+          if (hmask) hi = min(hi, r + delta + wr);
+          const int lo = (lmask ? r + delta - wl : 0) - half * 64;
+          hi -= half * 64;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
+          for (int c = 0; c < 64; ++c) s[c] = (c > hi || c < lo) ? -INFINITY : s[c];
         }
 #pragma unroll
         for (int c = 0; c < 64; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
@@ -423,10 +436,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (named_bar_and(5, 256, ok) && threadIdx.x == 0) {
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        tma_store_3d(&tmO, sbase + Lay::kK + c * Lay::kChunkBytes, c * 64, t * kTile, bh);
+        tma_store_4d(&tmO, sbase + Lay::kK + c * Lay::kChunkBytes, c * 64, t * kTile, hh, bb);
         if (has_res)
-          tma_store_3d(&tmOres, sbase + Lay::kK + Lay::kTileBytes + c * Lay::kChunkBytes, c * 64,
-                       t * kTile, bh);
+          tma_store_4d(&tmOres, sbase + Lay::kK + Lay::kTileBytes + c * Lay::kChunkBytes, c * 64,
+                       t * kTile, hh, bb);
       }
       bulk_commit();
       bulk_wait_read_all();  // shared memory is read before the CTA releases it

@@ -15,13 +15,22 @@
  * recomputes the scores from Q, K, V and uses L (josueisai.com, section "Recomputar
  * sale mas barato que recordar").
  *
- * Causal mask (optional; not on the pages): key j is visible to query i iff j <= i,
- * top-left aligned, N_q = N_k = N.
+ * Masks (not on the pages). Every mask is a key window around the bottom-right
+ * diagonal: with off = N_k - N_q, query i sees key j iff
+ *     i + off - window_left <= j <= i + off + window_right,
+ * a negative edge bounding nothing. (-1, -1) is unmasked attention, (-1, 0) the causal
+ * mask (with N_q = N_k: j <= i), and bounded edges a sliding window, the combination
+ * josueisai.com "flash-attention", section "Que ganas y que no", names for very long
+ * sequences. The basic calls' `causal` flag is (-1, 0) when set, (-1, -1) otherwise.
+ * A query row that sees no key gets O = 0 and L = -inf and contributes nothing to
+ * the gradients.
  *
- * Layout. Every 16-bit tensor (Q, K, V, O, dO, dQ, dK, dV) is a dense row-major
- * [B][H][N][d] array of one element type (bf16 or fp16, the `dtype` argument), so
- * element (b, h, n, t) sits at ((b*H + h)*N + n)*d + t. L is fp32 [B][H][N], in
- * natural-log units of the scaled score: L_i = m_i + ln(sum_j exp(s_ij - m_i)).
+ * Layout. Every 16-bit tensor (Q, K, V, O, dO, dQ, dK, dV) is a dense row-major array
+ * of one element type (bf16 or fp16, the `dtype` argument), either [B][H][N][d]
+ * (FA_LAYOUT_BHND, the basic calls' layout: element (b, h, n, t) at
+ * ((b*H + h)*N + n)*d + t) or [B][N][H][d] (FA_LAYOUT_BNHD: ((b*N + n)*H + h)*d + t).
+ * L is fp32 [B][H][N] in both, in natural-log units of the scaled score:
+ * L_i = m_i + ln(sum_j exp(s_ij - m_i)).
  * Arithmetic is fp32 with 16-bit MMA operands (P and dS are rounded to `dtype`
  * before their products).
  *
@@ -34,14 +43,17 @@
  * memory in these calls; its only state is one device-side error word per device.
  *
  * Supported now: d in {64, 128}; any N >= 1 (the last 128-row tile of a head may be
- * partial); dtype bf16 or fp16; B*H*N with N rounded up to 128 below 2^31.
+ * partial); dtype bf16 or fp16; B*H*N with N rounded up to 128 below 2^31, and
+ * N_q + N_k <= 2^29.
  *
  * Errors are checked on the host before anything is enqueued and are returned as
  * codes (no exception, no abort, no fallback to another implementation):
  *   FA_ERR_INVALID      null pointer, negative size, misaligned pointer, a workspace
- *                       that is too small, or a non-finite / non-positive scale;
- *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, or B*H*roundup(N,128)
- *                       >= 2^31 (32-bit TMA coordinates and grid indices);
+ *                       that is too small, a non-finite / non-positive scale, or an
+ *                       unknown layout or stage;
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, B*H*roundup(N,128)
+ *                       >= 2^31 (32-bit TMA coordinates and grid indices), or
+ *                       N_q + N_k > 2^29;
  *   FA_ERR_CUDA         a CUDA runtime/driver call or a launch failed;
  *   FA_ERR_TIMEOUT      (from fa_get_device_status only) a kernel gave up a bounded
  *                       wait on the device and returned without finishing.
@@ -66,6 +78,16 @@ typedef enum {
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
 
+typedef enum { FA_LAYOUT_BHND = 0, FA_LAYOUT_BNHD = 1 } fa_layout;
+
+/* Stages of the backward, for fa_bwd_ex_stage (bit flags; FA_STAGE_ALL = fa_bwd_ex). */
+typedef enum {
+    FA_STAGE_PREPROCESS = 1,
+    FA_STAGE_DKDV = 2,
+    FA_STAGE_DQ = 4,
+    FA_STAGE_ALL = 7
+} fa_stage;
+
 /*
  * Forward. Reads Q, K, V [B][H][N][d]; writes O [B][H][N][d] (dtype) and
  * L [B][H][N] (fp32). One kernel launch.
@@ -89,6 +111,18 @@ int fa_fwd(const void *Q, const void *K, const void *V, void *O, void *O_res, fl
  */
 int fa_fwd_qk(const void *Q, const void *K, const void *V, void *O, void *O_res, float *L, int B,
               int H, int Nq, int Nk, int d, int causal, float scale, int dtype, void *stream);
+
+/*
+ * Forward, general form: Q, O, O_res [.., Nq, ..], K, V [.., Nk, ..] in `layout`
+ * (FA_LAYOUT_BHND or FA_LAYOUT_BNHD), L [B][H][Nq] fp32, the key window
+ * [window_left, window_right] described at the top of this file (negative = that side
+ * unbounded). Key tiles outside every row's window are neither loaded nor multiplied.
+ * fa_fwd_qk(..., causal, ...) is fa_fwd_ex(..., FA_LAYOUT_BHND, -1, causal ? 0 : -1,
+ * ...). One kernel launch.
+ */
+int fa_fwd_ex(const void *Q, const void *K, const void *V, void *O, void *O_res, float *L,
+              int B, int H, int Nq, int Nk, int d, int layout, int window_left,
+              int window_right, float scale, int dtype, void *stream);
 
 /*
  * Bytes of device workspace that fa_bwd needs for this shape: fp32 D and scaled L
@@ -122,6 +156,57 @@ int fa_bwd_qk(const void *Q, const void *K, const void *V, const void *O, const 
               const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, void *workspace,
               size_t workspace_bytes, void *stream);
+
+/*
+ * Backward, general form (shapes, layout and window as fa_fwd_ex; dQ and dO are
+ * [.., Nq, ..], dK and dV [.., Nk, ..]). With B*H*Nq == 0 and Nk > 0, dK and dV are set
+ * to zero. The workspace is sized by fa_bwd_ex_workspace_size with the same arguments.
+ *
+ * `deterministic` = 0: dQ partial sums of the key tiles are added into an fp32
+ * accumulator in the workspace by the dK/dV kernel, in whatever order its CTAs finish,
+ * so dQ may differ in its last bits between calls (dK, dV, O, L never do).
+ * `deterministic` = 1: dQ is formed by a separate pass over the keys (one CTA per query
+ * tile summing the key tiles of its band in increasing order, accumulating in tensor
+ * memory), so every result is identical on every call; the dK/dV kernel then skips its
+ * dQ work and the workspace holds only the row statistics (B*H*Np*8 bytes). It costs
+ * the recomputation of S and dP in the dQ pass. Other values: FA_ERR_INVALID.
+ */
+size_t fa_bwd_ex_workspace_size(int B, int H, int Nq, int Nk, int d, int deterministic);
+int fa_bwd_ex(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
+              const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H, int Nq,
+              int Nk, int d, int layout, int window_left, int window_right, int deterministic,
+              float scale, int dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The stages of fa_bwd_ex selected by the bit set `stages` (fa_stage), with the same
+ * arguments and checks; pointers that the selected stages do not read or write may be
+ * NULL. Running FA_STAGE_PREPROCESS, FA_STAGE_DKDV and FA_STAGE_DQ in this order on one
+ * stream is fa_bwd_ex; each stage is one kernel launch (bench.py times them one by
+ * one).
+ *   FA_STAGE_PREPROCESS  D_i = sum_t dO_it (O_it + O_res_it) and -L * log2(e) into the
+ *                        workspace, and zeroes its fp32 dQ accumulator (if any);
+ *   FA_STAGE_DKDV        recomputes P from Q, K and the workspace's scaled L, writes
+ *                        dK and dV, and adds the dQ partials into the accumulator;
+ *   FA_STAGE_DQ          dQ = dtype(scale * accumulator); in deterministic mode the
+ *                        separate dQ pass, which reads Q, K, V, dO and the workspace's
+ *                        row statistics.
+ */
+int fa_bwd_ex_stage(int stages, const void *Q, const void *K, const void *V, const void *O,
+                    const void *O_res, const void *dO, const float *L, void *dQ, void *dK,
+                    void *dV, int B, int H, int Nq, int Nk, int d, int layout, int window_left,
+                    int window_right, int deterministic, float scale, int dtype, void *workspace,
+                    size_t workspace_bytes, void *stream);
+
+/*
+ * The tile schedule of a key window, for callers that size or account for the work:
+ * with query_side = 1, the key/value tiles (of 128 keys) that query tile `tile` (rows
+ * 128*tile .. 128*tile + 127) visits in the forward; with query_side = 0, the query
+ * tiles that key tile `tile` visits in the dK/dV pass. Writes the first tile and the
+ * count (0: none) of a consecutive range. FA_ERR_INVALID for a tile out of range,
+ * non-positive lengths or a NULL output. Touches no device.
+ */
+int fa_tile_range(int query_side, int tile, int Nq, int Nk, int window_left, int window_right,
+                  int *first, int *count);
 
 /*
  * The three stages of fa_bwd, callable one by one (same arguments, same checks, same
@@ -173,6 +258,30 @@ int fa_bwd_dq_convert(void *dQ, int B, int H, int N, int d, float scale, int dty
 int fa_bwd_noalloc(const void *Q, const void *K, const void *V, const void *O, const void *O_res,
                    const void *dO, const float *L, void *dQ, void *dK, void *dV, int B, int H,
                    int N, int d, int causal, float scale, int dtype, void *stream);
+
+/*
+ * Decode: a few query rows (1 <= Nq <= 16 per head) against a long key sequence,
+ * forward only. Same operation, shapes, layouts and key window as fa_fwd_ex (with
+ * Nq <= 16 the bottom-right-aligned causal mask lets query i see keys j <= i + Nk - Nq);
+ * writes O and L. The keys of each head are cut into splits of 128-key tiles, one CTA
+ * per (head, split), each running the online softmax over its tiles; a second kernel
+ * merges the splits' partial outputs by their log-sum-exps (L = ln sum_s exp(L_s),
+ * O = sum_s exp(L_s - L) O_s), the recurrence of josueisai.com "flash-attention",
+ * section "El truco", applied to whole splits. The pass reads K and V once and is
+ * bound by HBM, so it runs on CUDA cores; P is not rounded to 16 bits.
+ *
+ * The split count depends only on B*H, Nq, Nk and the window (it is chosen for 148
+ * SMs), so results are the same bits on every call. `workspace` (device, 256-byte
+ * aligned, caller-owned) holds the splits' partial results: at least
+ * fa_decode_workspace_size(B, H, Nq, Nk, d, window_left, window_right) bytes, which
+ * is 0 when one split suffices (workspace may then be NULL). Nq > 16:
+ * FA_ERR_UNSUPPORTED (use fa_fwd_ex).
+ */
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d, int window_left,
+                                int window_right);
+int fa_decode(const void *Q, const void *K, const void *V, void *O, float *L, int B, int H,
+              int Nq, int Nk, int d, int layout, int window_left, int window_right, float scale,
+              int dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device error word of the

@@ -83,3 +83,18 @@ def test_timing_inputs_have_the_workload_structure():
     assert torch.equal(q, q2)
     norms = q.float().norm(dim=-1)[0]             # [H, N]
     assert ((norms > 40).sum(dim=1) == 10).all()  # ~8 * sqrt(64) vs ~sqrt(64)
+
+
+@pytest.mark.parametrize("nq,nk", [(4, 4), (7, 30), (30, 7), (128, 1000)])
+@pytest.mark.parametrize("window", [(-1, -1), (-1, 0), (3, 0), (0, 5), (10, -1), (0, 0)])
+def test_visible_pairs_counts_the_window(nq, nk, window):
+    import numpy as np
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    off = nk - nq
+    vis = np.ones((nq, nk), bool)
+    if window[0] >= 0:
+        vis &= j >= i + off - window[0]
+    if window[1] >= 0:
+        vis &= j <= i + off + window[1]
+    assert bench.visible_pairs(nq, nk, window) == int(vis.sum())
