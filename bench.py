@@ -563,7 +563,7 @@ def main():
         pg.barrier()
     clocks = sampler.stop()
     total_ms = t_start.elapsed_time(t_end)
-    per_kernel = {"fa_fwd_kernel": 0.0, "fa_bwd_pre_kernel": 0.0, "fa_bwd_main_kernel": 0.0,
+    per_kernel = {"fa_fwd_pp_kernel": 0.0, "fa_bwd_pre_kernel": 0.0, "fa_bwd_main_kernel": 0.0,
                   "fa_bwd_dq_kernel": 0.0}
     names = list(per_kernel)
     for ev in events:
@@ -582,14 +582,14 @@ def main():
     ms_step = total_ms / steps
     # fwd+bwd counted as 2.5 x fwd, literally as the target states it
     value = job_throughput(world, 2.5 * fwd_f, steps, total_ms)
-    fwd_ms = per_kernel["fa_fwd_kernel"] / steps
+    fwd_ms = per_kernel["fa_fwd_pp_kernel"] / steps
     bwd_ms = sum(per_kernel[n] for n in names[1:]) / steps
     peaks, peak_kind = load_peaks()
     peak_burst = float(peaks["bf16_tflops"])
     peak_sus = float(peaks.get("bf16_tflops_sustained", peak_burst))
 
     # dominant kernel: the largest share of the step
-    kflops = {"fa_fwd_kernel": fwd_f, "fa_bwd_main_kernel": bwd_f}
+    kflops = {"fa_fwd_pp_kernel": fwd_f, "fa_bwd_main_kernel": bwd_f}
     rows = B * H * N
     kbytes = {"fa_bwd_pre_kernel": rows * d * 2 * 3 + rows * 4 + rows * 8 + rows * d * 4,
               "fa_bwd_dq_kernel": rows * d * 4 + rows * d * 2}

@@ -69,7 +69,7 @@ def parse_ptxas_report(text: str) -> dict:
 # Kernels that move registers between warpgroups with setmaxnreg: their split adds up
 # to exactly this many registers per thread at launch, so the compiled kernel must use
 # exactly that many (the library also refuses to launch otherwise).
-FIXED_REGISTERS = {"fa_bwd_main_kernel": 128}
+FIXED_REGISTERS = {"fa_bwd_main_kernel": 128, "fa_fwd_pp_kernel": 168}
 
 
 def check_resources(report: dict) -> None:

@@ -1,5 +1,5 @@
 // fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor
-// maps, and kernel launches. All device work is in fa_fwd.cuh / fa_bwd.cuh.
+// maps, and kernel launches. All device work is in the .cuh kernels beside it.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -12,7 +12,7 @@
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
-#include "fa_fwd.cuh"
+#include "fa_fwd_pp.cuh"
 
 namespace fa {
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing will
@@ -146,17 +146,23 @@ template <int D, bool BAND, bool BF16>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int B,
                int H, int Nq, int Nk, Window w, float scale, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, BAND, BF16>;
+  auto kern = fa::fa_fwd_pp_kernel<D, BAND, BF16>;
   // At least 120 KB so that one CTA -- and one 512-column TMEM allocation -- sits on
   // each SM (two CTAs would serialise on the tensor-memory allocation anyway).
-  const int smem = fa::FwdLayout<D>::kBytes > 120 * 1024 ? fa::FwdLayout<D>::kBytes : 120 * 1024;
+  const int smem = fa::PpLayout<D>::kBytes > 120 * 1024 ? fa::PpLayout<D>::kBytes : 120 * 1024;
+  if (static_cast<size_t>(smem) > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
-  const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) *
-                        static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
-  kern<<<grid, fa::kFwdThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
-                                                 w.wr, scale * 1.4426950408889634074f);
+  // The kernel moves registers between warpgroups (setmaxnreg); its split adds up to
+  // exactly 168 registers per thread at launch (the build fails otherwise too).
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FA_ERR_CUDA;
+  if (attr.numRegs != fa::kPpLaunchRegs) return FA_ERR_UNSUPPORTED;
+  const unsigned pairs = static_cast<unsigned>(((Nq + fa::kTile - 1) / fa::kTile + 1) / 2);
+  const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) * pairs;
+  kern<<<grid, fa::kPpThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
+                                                w.wr, scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -384,19 +390,20 @@ size_t decode_workspace(long BH, int Nq, int d, int splits) {
   return splits <= 1 ? 0 : static_cast<size_t>(BH) * splits * Nq * (static_cast<size_t>(d) + 1) * 4;
 }
 
-template <int D, int NQ, bool BAND, bool BF16>
+template <int D, int QW, bool BAND, bool BF16>
 int launch_decode_nq(const CUtensorMap& k, const CUtensorMap& v, const void* Q,
                      const fa::Strides& sq, void* O, float* L, float* opart, float* lpart, int B,
                      int H, int Nq, int Nk, const Window& w, fa::TileRange tiles, int splits,
                      float scale, cudaStream_t stream) {
-  auto kern = fa::fa_decode_kernel<D, NQ, BAND, BF16>;
+  auto kern = fa::fa_decode_kernel<D, QW, BAND, BF16>;
   const int smem = fa::DecLayout<D>::kBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return FA_ERR_CUDA;
   const long BH = static_cast<long>(B) * H;
   const int tps = tiles.count > 0 ? (tiles.count + splits - 1) / splits : 0;
-  kern<<<static_cast<unsigned>(BH * splits), fa::dec_threads(NQ), smem, stream>>>(
+  const long groups = (Nq + fa::kDecQPerCta - 1) / fa::kDecQPerCta;
+  kern<<<static_cast<unsigned>(BH * splits * groups), fa::kDecThreads, smem, stream>>>(
       k, v, static_cast<const uint16_t*>(Q), sq, static_cast<uint16_t*>(O), sq, L, opart, lpart,
       Nq, Nk, H, w.wl, w.wr, tiles.first, tiles.count, tps, splits,
       scale * 1.4426950408889634074f);
@@ -416,7 +423,7 @@ struct DecodeRun {
   static int run(int Nq, A&&... a) {
     if (Nq <= 1) return launch_decode_nq<D, 1, BAND, BF16>(a...);
     if (Nq <= 4) return launch_decode_nq<D, 4, BAND, BF16>(a...);
-    return launch_decode_nq<D, 16, BAND, BF16>(a...);
+    return launch_decode_nq<D, 8, BAND, BF16>(a...);  // 8 rows per CTA
   }
 };
 
@@ -609,7 +616,7 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
   if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
                    workspace_bytes < need))
     return FA_ERR_INVALID;
-  if (BH * splits >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  if (BH * splits * 2 >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tk, tv;
   if (!make_tmap(&tk, K, B, H, Nk, d, layout, dtype) ||
       !make_tmap(&tv, V, B, H, Nk, d, layout, dtype))

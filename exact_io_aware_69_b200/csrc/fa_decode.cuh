@@ -13,9 +13,9 @@
 // "FlashAttention" names inference serving as a user of the method; foqum.io
 // "FlashAttention", Q3, the long contexts it makes affordable.)
 //
-// CTA: 4 compute warps per group of up to 8 query rows (8 warps for 9-16 rows) and 1
-// TMA producer warp. Warp w takes keys 32 (w % 4) .. 32 (w % 4) + 31 of every tile and
-// the query rows of its group. For the scores each lane owns d/32 columns: it forms 32 partial dot
+// CTA: 4 compute warps and 1 TMA producer warp, for up to 8 query rows (rows 9-16 of a
+// head go to a second CTA over the same keys, whose tiles then mostly come from L2).
+// Warp w takes keys 32 w .. 32 w + 31 of every tile. For the scores each lane owns d/32 columns: it forms 32 partial dot
 // products (one per key of the warp's group) and a butterfly reduce-scatter over the
 // lanes leaves lane k with the full score of key k. For P V each lane owns the same
 // d/32 columns of O and takes the probabilities from the key lanes by shuffle. Each
@@ -28,14 +28,10 @@
 
 namespace fa {
 
-constexpr int kDecWarps = 4;    // compute warps per query group (one per 32 keys of a tile)
+constexpr int kDecWarps = 4;     // compute warps (one per 32 keys of a tile)
+constexpr int kDecThreads = (kDecWarps + 1) * 32;  // + the TMA producer warp
 constexpr int kDecMaxQ = 16;
-constexpr int kDecQPerWarp = 8;  // query rows one warp carries
-// Query groups for NQ rows: warps 4g .. 4g + 3 carry rows [8g, 8g + 8).
-__host__ __device__ constexpr int dec_groups(int nq) {
-  return nq > kDecQPerWarp ? (nq + kDecQPerWarp - 1) / kDecQPerWarp : 1;
-}
-__host__ __device__ constexpr int dec_threads(int nq) { return (kDecWarps * dec_groups(nq) + 1) * 32; }
+constexpr int kDecQPerCta = 8;   // query rows one CTA carries; 9-16 rows take two CTAs
 
 template <int D>
 struct DecLayout {
@@ -108,12 +104,13 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// One CTA per (head bh, split s); the split covers key tiles [tile0 + s*tps,
-// min(tile0 + ntiles, tile0 + (s+1)*tps)). With splits == 1 the CTA writes O (16-bit,
-// strides so) and L itself; otherwise its normalised partial output and log-sum-exp
-// go to Opart [BH][splits][Nq][D] and Lpart [BH][splits][Nq] (fp32) for the merge.
-template <int D, int NQ, bool BAND, bool BF16>
-__global__ void __maxnreg__(224)
+// One CTA per (head bh, split s, query group); the split covers key tiles
+// [tile0 + s*tps, min(tile0 + ntiles, tile0 + (s+1)*tps)), the group query rows
+// [8 group, 8 group + QW). With splits == 1 the CTA writes O (16-bit, strides so) and L
+// itself; otherwise its normalised partial output and log-sum-exp go to Opart
+// [BH][splits][Nq][D] and Lpart [BH][splits][Nq] (fp32) for the merge.
+template <int D, int QW, bool BAND, bool BF16>
+__global__ void __launch_bounds__(kDecThreads, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const uint16_t* __restrict__ Q,
                      Strides sq, uint16_t* __restrict__ O, Strides so, float* __restrict__ Lse,
@@ -123,9 +120,7 @@ __global__ void __maxnreg__(224)
   using Lay = DecLayout<D>;
   constexpr int CPL = D / 32;  // columns per lane
   constexpr int S = Lay::kStages;
-  constexpr int G = dec_groups(NQ);
-  constexpr int QW = NQ / G;             // query rows per warp
-  constexpr int kCompute = kDecWarps * G;  // compute warps
+  constexpr int kCompute = kDecWarps;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
@@ -134,8 +129,11 @@ __global__ void __maxnreg__(224)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x / splits;
-  const int sp = blockIdx.x - bh * splits;
+  const int groups = (Nq + kDecQPerCta - 1) / kDecQPerCta;
+  const int cta = blockIdx.x / groups;  // (head, split)
+  const int grp = blockIdx.x - cta * groups;
+  const int bh = cta / splits;
+  const int sp = cta - bh * splits;
   const int hh = bh % H;
   const int bb = bh / H;
   const int t_begin = tile0 + sp * tps;
@@ -179,8 +177,8 @@ __global__ void __maxnreg__(224)
   }
 
   // ------------------------------------------------------------------- compute
-  const int kw = warp % kDecWarps;  // key group: rows 32 kw .. 32 kw + 31 of every tile
-  const int q0 = (warp / kDecWarps) * QW;  // first query row of this warp's group
+  const int kw = warp;            // key group: rows 32 kw .. 32 kw + 31 of every tile
+  const int q0 = grp * kDecQPerCta;  // first query row of this CTA
   // this lane's columns of the group's query rows, times scale * log2(e): scores come
   // out in base-2 units
   float qr[QW][CPL];
@@ -265,8 +263,8 @@ __global__ void __maxnreg__(224)
     if (lane == 0) mbar_arrive(empty(st));
   }
 
-  // merge the four key groups' (m, l, O) of every row, in the ring (every warp is past
-  // its last tile)
+  // merge the four key groups' (m, l, O) of every row of this CTA, in the ring (every
+  // warp is past its last tile)
   const bool all_ok = named_bar_and(1, kCompute * 32, ok);
   float* wm = reinterpret_cast<float*>(smem);           // [key group][row]
   float* wsum = wm + kDecWarps * kDecMaxQ;               // [key group][row]
@@ -286,7 +284,8 @@ __global__ void __maxnreg__(224)
   }
   named_bar_sync(1, kCompute * 32);
   if (!all_ok) return;
-  for (int q = warp; q < Nq; q += kCompute) {
+  const int q_end = min(Nq, q0 + QW);
+  for (int q = q0 + warp; q < q_end; q += kCompute) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, wm[w * kDecMaxQ + q]);

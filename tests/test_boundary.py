@@ -341,3 +341,28 @@ def test_decode_rejects_before_launch(lib):
     assert call(Nk=1 << 20, ws_bytes=16) == fa.FA_ERR_INVALID
     assert call(Nk=1 << 20, ws=P + 0x900010) == fa.FA_ERR_INVALID  # 256-byte alignment
     assert call(Nq=0) == fa.FA_OK
+
+
+# Threads per block of every kernel the library launches.
+BLOCK_THREADS = {"fa_fwd_pp_kernel": 384, "fa_bwd_main_kernel": 512, "fa_bwd_dq_pass_kernel": 320,
+                 "fa_decode_kernel": 160, "fa_decode_merge_kernel": 256,
+                 "fa_bwd_pre_kernel": 256, "fa_bwd_dq_kernel": 256,
+                 "fa_selftest_wait_kernel": 32}
+
+
+def test_every_kernel_fits_the_register_file_at_its_block_size():
+    """A block whose warps need more registers than a sub-partition holds (16,384: each
+    of the SM's 4 sub-partitions runs every 4th warp) is refused at launch. Check each
+    compiled kernel against the block size the library launches it with."""
+    rep = build.resources()
+    seen = set()
+    for name, res in rep.items():
+        fam = [k for k in BLOCK_THREADS if k in name]
+        assert len(fam) == 1, name
+        seen.add(fam[0])
+        warps = -(-BLOCK_THREADS[fam[0]] // 32)
+        per_sub = -(-warps // 4)
+        regs = -(-res["registers"] // 8) * 8  # allocated in units of 8 per thread
+        assert regs * 32 * per_sub <= 16384, (name, res["registers"], BLOCK_THREADS[fam[0]])
+        assert res["spill_stores"] <= 8, (name, res)
+    assert seen == set(BLOCK_THREADS)
