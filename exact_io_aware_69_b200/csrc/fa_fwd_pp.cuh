@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_base + pad;
 
+  FA_TRACE_CTA(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  FA_TRACE_BEGIN();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Lay::kTmemSlot);
 
@@ -202,6 +204,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sbase + Lay::kK + ks * Lay::kTileBytes + c * Lay::kChunkBytes, &tmK,
                         c * 64, (J0 + step) * kTile, hh, bb, bar(kPbKFull + ks));
+          FA_TRACE_EVENT(step, 10);
         }
         if (step >= 1) {
           const int i = step - 1;
@@ -214,6 +217,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sbase + Lay::kV + vs * Lay::kTileBytes + c * Lay::kChunkBytes, &tmV,
                         c * 64, (J0 + i) * kTile, hh, bb, bar(kPbVFull + vs));
+          FA_TRACE_EVENT(i, 11);
         }
       }
     }
@@ -254,6 +258,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
               mma_ts(d_o, a_p + k * 8, sdesc_step(dv, k * 2048), idesc_o,
                      (u > 0 || k > 0) ? 1u : 0u);
             if (j == first_of(g) + count_of(g)) mma_commit(bar(kPbODone + g));  // its last P V
+            FA_TRACE_EVENT(i, 2 * g);
           }
           if (in_range(g, j)) {  // S_g,j = Q_g K_j^T
             const int ks = i % kPpKStages;
@@ -274,6 +279,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                      idesc_s, k > 0 ? 1u : 0u);
             }
             mma_commit(bar(kPbSFull + g));
+            FA_TRACE_EVENT(i, 2 * g + 1);
           }
         }
         if (!ok) break;
@@ -303,6 +309,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bar(kPbSFull + g), static_cast<uint32_t>(u) & 1, abort_flag));
       if (!ok) break;
+      if (r == 0) FA_TRACE_EVENT(u, 4 + 3 * g);
       tc_fence_after();
       float s[128];
       {
@@ -337,6 +344,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         for (int k = 0; k < 4; ++k) mq[k] = fmax3(mq[k], s[c + 2 * k], s[c + 2 * k + 1]);
       }
       const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      if (r == 0) FA_TRACE_EVENT(u, 5 + 3 * g);
       const float cand = mx * scale_log2;
       const float m_new = (cand > m + kPpRescaleSlack) ? cand : m;
       // A row that sees no key keeps m = -inf: it takes alpha = 1 and subtracts 0, so
@@ -389,6 +397,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kPbPFull + g));
+      if (r == 0) FA_TRACE_EVENT(u, 6 + 3 * g);
       m = m_new;
     }
     // epilogue: O / l_o and O's rounding residual, staged in this warpgroup's Q tile
@@ -480,6 +489,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  FA_TRACE_CTA(1);
 }
 
 }  // namespace fa
