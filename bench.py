@@ -275,6 +275,32 @@ def time_workload(fa, w, dev, stream, steps, warmup, peak_burst, window=None, la
     return r
 
 
+def time_forward(fa, w, dev, stream, steps, warmup, peak_burst):
+    """Device time per forward of workload w alone (for head dimensions the backward does
+    not take), CUDA events on the launching stream."""
+    import torch
+    q, k, v, _ = torch_inputs(w, dev, w.seed)
+    o, o_res = torch.empty_like(q), torch.empty_like(q)
+    L = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        fa.forward(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=L, out_res=o_res,
+                   stream=stream)
+    e0.record(stream)
+    for _ in range(steps):
+        fa.forward(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=L, out_res=o_res,
+                   stream=stream)
+    e1.record(stream)
+    e1.synchronize()
+    st = fa.device_status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"device status {st} in {w.name}")
+    ms = e0.elapsed_time(e1) / steps
+    f, _ = flops(w)
+    return {"fwd_ms": round(ms, 4), "fwd_tflops": round(f / ms / 1e9, 1),
+            "frac_of_burst": round(f / ms / 1e9 / peak_burst, 3)}
+
+
 def time_decode(fa, B, H, Nq, Nk, d, dev, stream, steps, warmup, hbm_peak):
     """The split-KV decode path: Nq rows per head against Nk keys, causal. Its bound is
     HBM: K and V are read once (plus Q, O, L), so the rate is reported in GB/s."""
@@ -707,6 +733,11 @@ def main():
                                                     layout="bnhd")
         by_w["c3 deterministic backward"] = time_workload(fa, c3, dev, stream, 5, 3, peak_burst,
                                                           deterministic=True)
+        # head dimension 256 (forward only)
+        for causal in (True, False):
+            w256 = type(c3)(f"B2 H16 N8192 d256 bf16 {'causal' if causal else 'non-causal'}, "
+                            "forward only", 2, 16, 8192, 256, "bf16", causal, 8256 + causal)
+            by_w[w256.name] = time_forward(fa, w256, dev, stream, 5, 3, peak_burst)
         extras["by_workload"] = by_w
         hbm = float(peaks["hbm_gbs"])
         extras["decode"] = [time_decode(fa, 4, 32, nq, 65536, 128, dev, stream, 10, 3, hbm)

@@ -12,6 +12,7 @@
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
+#include "fa_fwd_d256.cuh"
 #include "fa_fwd_pp.cuh"
 
 namespace fa {
@@ -27,6 +28,18 @@ __global__ void fa_selftest_wait_kernel(long long limit_cycles) {
   mbar_init(smem_u32(&bar), 1);
   fence_mbar_init();
   mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_cycles);
+}
+
+// Self-test of the forward's FMA-pipe exponential: y = ex2_poly_pair(x) elementwise
+// (n even), so that it can be held against CUDA's exp2f.
+__global__ void fa_selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                        int npairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= npairs) return;
+  float y0, y1;
+  ex2_poly_pair(x[2 * i], x[2 * i + 1], y0, y1);
+  y[2 * i] = y0;
+  y[2 * i + 1] = y1;
 }
 }  // namespace fa
 
@@ -105,13 +118,13 @@ bool ok_ptr(const void* p) { return p && aligned16(p); }
 // dK = dV = 0 when Nk > 0). Keys are required when there are queries: a row with no
 // key at all has no softmax.
 int check_shape(int B, int H, int Nq, int Nk, int d, int layout, int dtype, float scale,
-                bool* empty) {
+                bool* empty, bool d256_ok = false) {
   *empty = false;
   if (B < 0 || H < 0 || Nq < 0 || Nk < 0 || d < 0) return FA_ERR_INVALID;
   if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BNHD) return FA_ERR_INVALID;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_UNSUPPORTED;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && !(d256_ok && d == 256)) return FA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H * Nq == 0) {
     *empty = true;
     return FA_OK;
@@ -163,6 +176,24 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) * pairs;
   kern<<<grid, fa::kPpThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
                                                 w.wr, scale * 1.4426950408889634074f);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// d = 256: one query tile per CTA (fa_fwd_d256.cuh).
+template <bool BAND, bool BF16>
+int launch_fwd_d256(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                    const CUtensorMap& o, const CUtensorMap& o_res, bool has_res, float* L, int B,
+                    int H, int Nq, int Nk, Window w, float scale, cudaStream_t stream) {
+  auto kern = fa::fa_fwd_d256_kernel<BAND, BF16>;
+  const int smem = static_cast<int>(fa::WideLayout::kBytes);
+  if (static_cast<size_t>(smem) > kMaxDynSmem) return FA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  const unsigned tiles = static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
+  const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) * tiles;
+  kern<<<grid, fa::kWThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
+                                              w.wr, scale * 1.4426950408889634074f);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -471,7 +502,7 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, void* O_res,
               int B, int H, int Nq, int Nk, int d, int layout, int window_left,
               int window_right, float scale, int dtype, void* stream) {
   bool empty;
-  int st = check_shape(B, H, Nq, Nk, d, layout, dtype, scale, &empty);
+  int st = check_shape(B, H, Nq, Nk, d, layout, dtype, scale, &empty, /*d256_ok=*/true);
   if (st != FA_OK || empty) return st;
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(O) || !ok_ptr(L) || !aligned16(O_res))
     return FA_ERR_INVALID;
@@ -483,8 +514,21 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, void* O_res,
       !make_tmap(&tr, O_res != nullptr ? O_res : O, B, H, Nq, d, layout, dtype))
     return FA_ERR_CUDA;
   const Window w = window_of(Nq, Nk, window_left, window_right);
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (d == 256) {
+    const bool bf = dtype == FA_BF16;
+    if (w.band)
+      return bf ? launch_fwd_d256<true, true>(tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
+                                              Nk, w, scale, cs)
+                : launch_fwd_d256<true, false>(tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
+                                               Nk, w, scale, cs);
+    return bf ? launch_fwd_d256<false, true>(tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
+                                             Nk, w, scale, cs)
+              : launch_fwd_d256<false, false>(tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
+                                              Nk, w, scale, cs);
+  }
   return dispatch<FwdRun>(d, w.band, dtype, tq, tk, tv, to, tr, O_res != nullptr, L, B, H, Nq,
-                          Nk, w, scale, static_cast<cudaStream_t>(stream));
+                          Nk, w, scale, cs);
 }
 
 int fa_fwd_qk(const void* Q, const void* K, const void* V, void* O, void* O_res, float* L,
@@ -652,6 +696,18 @@ int fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
 int fa_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles <= 0 || limit_cycles > fa::kWaitLimitCycles) return FA_ERR_INVALID;
   fa::fa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n & 1)) return FA_ERR_INVALID;
+  if (n == 0) return FA_OK;
+  if (x == nullptr || y == nullptr || (reinterpret_cast<uintptr_t>(x) & 7) ||
+      (reinterpret_cast<uintptr_t>(y) & 7))
+    return FA_ERR_INVALID;
+  const int npairs = n / 2;
+  fa::fa_selftest_exp2_kernel<<<(npairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, y, npairs);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -27,7 +27,9 @@
 //              takes query columns 0-63, warp w+4 columns 64-127 (no row reduction
 //              is needed here: L and D are per query column). P^T from S^T and L,
 //              dS^T from dP^T and D; P^T goes back to TMEM (16-bit), dS^T to shared
-//              memory (16-bit, 128-byte swizzle) for two MMAs; at the end the
+//              memory (16-bit, 128-byte swizzle; the dQ MMA's A, read M-major, which
+//              TMEM cannot give) and at d = 128 also to TMEM (16-bit, over dP^T
+//              columns already read; the dK MMA's A); at the end the
 //              dK_j / dV_j epilogue, each warp of the pair writing half the columns.
 //   warps 8-11 dQ drain (200 registers each): thread owns query row (warp % 4) * 32 +
 //              lane; takes the whole dQ_i row out of TMEM at once, so that the
@@ -40,7 +42,8 @@
 //   warp 13    MMA issuer (and TMEM owner), per query tile:
 //                S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (SMEM x SMEM)
 //                dV += P^T dO_i                              (P^T from TMEM)
-//                dK += dS^T Q_i, dQ_i = dS K_j                (dS from SMEM)
+//                dK += dS^T Q_i                   (dS^T from TMEM at d = 128)
+//                dQ_i = dS K_j                               (dS from SMEM)
 //   warps 14-15 idle (they complete warpgroup 3, which runs on 56 registers).
 #pragma once
 
@@ -199,6 +202,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int Nq, int Nk,
                        int H, int wl, int wr, Strides kv, float scale, float scale_log2,
                        uint32_t smem_alloc) {
+  // dS^T for the dK MMA: from TMEM at d = 128, from shared memory at d = 64
+  constexpr bool kDsInTmem = D == 128;
   using Lay = BwdLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -378,13 +383,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         FA_TRACE_EVENT(it, 1);
         if (DQ && D != 128 && it > 0 && !mbar_wait(bar(kBbDQEmpty), ph ^ 1u, abort_flag)) break;
         tc_fence_after();
-        // dK += dS^T Q_i
+        // dK += dS^T Q_i. At d = 128 dS^T comes from TMEM: query columns 16k .. 16k + 15
+        // are packed in the dP^T columns of the compute warp that owns them (64 per half,
+        // the first 32 used); at d = 64 from shared memory.
         const uint64_t dq_mn = sdesc_sw128(sq, Lay::kChunkBytes, 1024);
 #pragma unroll
         for (int k = 0; k < kTile / 16; ++k) {
-          const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
-          mma_ss(tmem + Lay::tDK, sdesc_step(dds_k, koff), sdesc_step(dq_mn, k * 2048), id_acc,
-                 (it > 0 || k > 0) ? 1u : 0u);
+          if constexpr (kDsInTmem) {
+            mma_ts(tmem + Lay::tDK, tmem + Lay::tDP + (k >> 2) * 64 + (k & 3) * 8,
+                   sdesc_step(dq_mn, k * 2048), id_acc, (it > 0 || k > 0) ? 1u : 0u);
+          } else {
+            const uint32_t koff = (k >> 2) * Lay::kChunkBytes + (k & 3) * 32;
+            mma_ss(tmem + Lay::tDK, sdesc_step(dds_k, koff), sdesc_step(dq_mn, k * 2048), id_acc,
+                   (it > 0 || k > 0) ? 1u : 0u);
+          }
         }
         if constexpr (DQ) {
           // dQ_i = dS K_j   (dS read M-major from the same shared tile)
@@ -515,11 +527,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           const int unit = (c * 4 + u) ^ sw;
           *reinterpret_cast<uint4*>(sds_row + unit * 16) = make_uint4(ds[0], ds[1], ds[2], ds[3]);
+          // at d = 128 the same 8 query columns also go to tensor memory, packed over
+          // dP^T columns this warp has loaded already (the first 32 of its 64): the dK
+          // MMA takes its A operand from there and reads no shared memory for it (at
+          // d = 64 the kernel has shared-memory bandwidth to spare, and the extra live
+          // values would spill in its band variants)
+          if constexpr (kDsInTmem)
+            tmem_st4(lane_base + Lay::tDP + half * 64 + c * 16 + 4 * u, ds[0], ds[1], ds[2],
+                     ds[3]);
         }
       }
       fence_async_smem();
+      if constexpr (kDsInTmem) tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBbDSReady));  // dS^T is in shared memory: dK and dQ may go
+      mbar_arrive(bar(kBbDSReady));  // dS^T is in place: dK and dQ may go
       if (threadIdx.x == 0) FA_TRACE_EVENT(it, 11);
     }
     // A key tile that no query sees (possible under a sliding window) ran no MMA: its

@@ -43,6 +43,8 @@
 // backward uses it for D = rowsum(dO * O).
 #pragma once
 
+#include <type_traits>
+
 #include "fa_band.cuh"
 #include "sm100.cuh"
 
@@ -59,6 +61,15 @@ constexpr int kPpSoftmaxRegs = 224;
 constexpr int kPpSmallRegs = 56;
 static_assert(2 * kPpSoftmaxRegs + kPpSmallRegs == 3 * kPpLaunchRegs, "register split");
 constexpr float kPpRescaleSlack = 8.0f;
+// Of every 16 exponential pairs of a softmax thread, how many go to the FMA pipe on
+// tiles without a mask (a power of two up to 16; 0 = MUFU only).
+#ifndef FA_PP_POLY_PAIRS
+#define FA_PP_POLY_PAIRS 2
+#endif
+constexpr int kPpPolyPairs = FA_PP_POLY_PAIRS;
+static_assert(kPpPolyPairs >= 0 && kPpPolyPairs <= 16 && (kPpPolyPairs & (kPpPolyPairs - 1)) == 0,
+              "poly pairs");
+constexpr int kPpPolyStride = kPpPolyPairs > 0 ? 16 / kPpPolyPairs : 16;
 constexpr int kPpKStages = 3;
 constexpr int kPpVStages = 2;
 
@@ -355,26 +366,42 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
       // packed fp32 pairs, two independent accumulators per sum (16-deep chains)
       uint64_t sum2[2] = {0, 0}, sum2_o[2] = {0, 0};  // packed +0.0f
+      // Exponentials on MUFU; on tiles without a mask, kPpPolyPairs of every 16 pairs
+      // on the FMA pipe instead (ex2_poly_pair), which shortens a warp's exponential
+      // phase when it has its sub-partition's MUFU to itself. Masked tiles stay on
+      // MUFU, which returns exact zeros for masked scores.
+      auto exps = [&](auto poly_tag) {
+        constexpr bool kPoly = decltype(poly_tag)::value;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t pk[16];
+        for (int h = 0; h < 4; ++h) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int e = h * 32 + 2 * c;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nm2), x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          pk[c] = pack2<BF16>(p0, p1);
-          float r0, r1;
-          unpack2<BF16>(pk[c], r0, r1);
-          sum2[c & 1] = f2_add(sum2[c & 1], f2_pack(p0, p1));
-          sum2_o[c & 1] = f2_add(sum2_o[c & 1], f2_pack(r0, r1));
+          for (int c = 0; c < 16; ++c) {
+            const int e = h * 32 + 2 * c;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nm2), x0, x1);
+            float p0, p1;
+            if (kPoly && c % kPpPolyStride == kPpPolyStride - 1) {
+              ex2_poly_pair(x0, x1, p0, p1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            pk[c] = pack2<BF16>(p0, p1);
+            float r0, r1;
+            unpack2<BF16>(pk[c], r0, r1);
+            sum2[c & 1] = f2_add(sum2[c & 1], f2_pack(p0, p1));
+            sum2_o[c & 1] = f2_add(sum2_o[c & 1], f2_pack(r0, r1));
+          }
+          // P packed over the first 64 columns of the S buffer; this thread owns the
+          // row, and all of S is in registers already
+          tmem_st16(lane_base + s_cols + h * 16, pk);
         }
-        // P packed over the first 64 columns of the S buffer; this thread owns the row,
-        // and all of S is in registers already
-        tmem_st16(lane_base + s_cols + h * 16, pk);
-      }
+      };
+      if (kPpPolyPairs > 0 && !(hmask || lmask || kmask))
+        exps(std::integral_constant<bool, true>{});
+      else
+        exps(std::integral_constant<bool, false>{});
       float a0, a1, b0, b1;
       f2_unpack(f2_add(sum2[0], sum2[1]), a0, a1);
       f2_unpack(f2_add(sum2_o[0], sum2_o[1]), b0, b1);

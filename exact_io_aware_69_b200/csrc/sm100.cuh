@@ -312,6 +312,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// Four consecutive 32-bit columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                         uint32_t r3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0),
+               "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 // --------------------------------------------------------- MMA descriptors
 // Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes with
 // CU_TENSOR_MAP_SWIZZLE_128B): start address, leading- and stride-dimension byte
@@ -444,6 +452,38 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// 2^x for a pair of arguments on the FMA and integer pipes, without the MUFU unit, so
+// that a softmax can split its exponentials between the two. Argument split in the
+// manner of Cody and Waite ("Software Manual for the Elementary Functions", 1980):
+// x = i + f with i = round(x), which the sum x + 1.5 * 2^23 holds in its low mantissa
+// bits, and f = x - i in [-1/2, 1/2] exactly. 2^f is the degree-4 minimax polynomial
+// (relative error) fitted by the Remez exchange in exact_io_aware_69_b200/fit_exp2.py:
+// max relative error 2.7e-6 in this float32 evaluation, far below the 2^-9 / 2^-11
+// rounding of the 16-bit P it feeds. 2^i is added into the exponent field: the bits
+// of the shifted sum, shifted left by 23, equal i << 23 modulo 2^32. Arguments below
+// -125 are clamped, so the result is never 0 (2^-125 at least): callers keep exact
+// zeros, such as masked scores, on the MUFU path.
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.240247443318367f;
+constexpr float kExp2C3 = 0.05591785907745361f;
+constexpr float kExp2C4 = 0.009570102207362652f;
+__device__ __forceinline__ void ex2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(12582912.f, 12582912.f));
+  const uint64_t i = f2_add(t, f2_pack(-12582912.f, -12582912.f));  // round(x), exact
+  const uint64_t f = f2_fma(i, f2_pack(-1.f, -1.f), x);               // x - i, exact
+  uint64_t p = f2_fma(f2_pack(kExp2C4, kExp2C4), f, f2_pack(kExp2C3, kExp2C3));
+  p = f2_fma(p, f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // max of three
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

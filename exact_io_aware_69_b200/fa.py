@@ -60,6 +60,7 @@ SIGNATURES = {
     "fa_decode": (_int, [_vp] * 5 + [_int] * 8 + [_f32, _int, _vp, _sz, _vp]),
     "fa_get_device_status": (_int, [_vp]),
     "fa_selftest_wait_timeout": (_int, [ctypes.c_longlong, _vp]),
+    "fa_selftest_exp2": (_int, [_vp, _vp, _int, _vp]),
     "fa_status_string": (ctypes.c_char_p, [_int]),
     "fa_version": (_int, []),
 }

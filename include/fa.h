@@ -42,8 +42,10 @@
  * workspace sized by fa_bwd_workspace_size(). The library allocates no device
  * memory in these calls; its only state is one device-side error word per device.
  *
- * Supported now: d in {64, 128}; any N >= 1 (the last 128-row tile of a head may be
- * partial); dtype bf16 or fp16; B*H*N with N rounded up to 128 below 2^31, and
+ * Supported now: d in {64, 128} for every call, and d = 256 for the forward calls
+ * (fa_fwd, fa_fwd_qk, fa_fwd_ex: one query tile per CTA, its score buffers and O
+ * filling the 512 tensor-memory columns); any N >= 1 (the last 128-row tile of a head
+ * may be partial); dtype bf16 or fp16; B*H*N with N rounded up to 128 below 2^31, and
  * N_q + N_k <= 2^29.
  *
  * Errors are checked on the host before anything is enqueued and are returned as
@@ -51,7 +53,8 @@
  *   FA_ERR_INVALID      null pointer, negative size, misaligned pointer, a workspace
  *                       that is too small, a non-finite / non-positive scale, or an
  *                       unknown layout or stage;
- *   FA_ERR_UNSUPPORTED  d not in {64, 128}, dtype not bf16/fp16, B*H*roundup(N,128)
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128} (forward calls: {64, 128, 256}), dtype not
+ *                       bf16/fp16, B*H*roundup(N,128)
  *                       >= 2^31 (32-bit TMA coordinates and grid indices), or
  *                       N_q + N_k > 2^29;
  *   FA_ERR_CUDA         a CUDA runtime/driver call or a launch failed;
@@ -300,6 +303,17 @@ int fa_get_device_status(void *stream);
  * for a limit out of range.
  */
 int fa_selftest_wait_timeout(long long limit_cycles, void *stream);
+
+/*
+ * Self-test of the forward kernel's exponential on the FMA pipe (part of each softmax
+ * thread's 2^x is computed without the MUFU unit: a Cody-Waite style split x = i + f
+ * and a minimax polynomial for 2^f on [-1/2, 1/2]). Writes y[k] = that 2^x[k] for
+ * k < n, asynchronously on `stream`. x and y: device float arrays of n elements,
+ * 8-byte aligned, owned by the caller. n must be even; n = 0 returns FA_OK without a
+ * launch. FA_ERR_INVALID for a negative or odd n, a null or misaligned pointer.
+ * Inputs below -125 give 2^-125 (the kernel keeps masked scores off this path).
+ */
+int fa_selftest_exp2(const float *x, float *y, int n, void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *fa_status_string(int status);

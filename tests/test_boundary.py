@@ -26,7 +26,7 @@ def lib():
 def _declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():
@@ -34,7 +34,7 @@ def test_header_declares_the_boundary():
     assert names == sorted(["fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_get_device_status",
                             "fa_status_string", "fa_version", "fa_bwd_preprocess",
                             "fa_bwd_dkdv", "fa_bwd_dq_convert", "fa_bwd_noalloc",
-                            "fa_selftest_wait_timeout", "fa_fwd_qk", "fa_bwd_qk", "fa_fwd_ex",
+                            "fa_selftest_wait_timeout", "fa_selftest_exp2", "fa_fwd_qk", "fa_bwd_qk", "fa_fwd_ex",
                             "fa_bwd_ex", "fa_bwd_ex_stage", "fa_bwd_ex_workspace_size",
                             "fa_tile_range", "fa_decode", "fa_decode_workspace_size"])
 
@@ -95,7 +95,10 @@ def _bwd(lib, **kw):
     (dict(scale=float("nan")), fa.FA_ERR_INVALID),
     (dict(scale=float("inf")), fa.FA_ERR_INVALID),
     (dict(d=96), fa.FA_ERR_UNSUPPORTED),
-    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=192), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=512), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256, B=0), fa.FA_OK),               # d = 256 passes the shape checks ...
+    (dict(d=256, K=P + 8), fa.FA_ERR_INVALID),  # ... and reaches the pointer checks
     (dict(B=1 << 15, H=1 << 10, N=100), fa.FA_ERR_UNSUPPORTED),  # 2^32 padded rows
     (dict(dtype=2), fa.FA_ERR_UNSUPPORTED),
     (dict(B=0), fa.FA_OK),
@@ -114,6 +117,7 @@ def test_fwd_rejects_before_launch(lib, kw, code):
     (dict(R=P + 0xa00008), fa.FA_ERR_INVALID),
     (dict(H=-2), fa.FA_ERR_INVALID),
     (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),  # the backward has no d = 256 kernel
     (dict(B=1 << 20, H=16, N=130), fa.FA_ERR_UNSUPPORTED),  # 2^32 padded rows
     (dict(dtype=5), fa.FA_ERR_UNSUPPORTED),
     (dict(H=0), fa.FA_OK),
@@ -345,9 +349,9 @@ def test_decode_rejects_before_launch(lib):
 
 # Threads per block of every kernel the library launches.
 BLOCK_THREADS = {"fa_fwd_pp_kernel": 384, "fa_bwd_main_kernel": 512, "fa_bwd_dq_pass_kernel": 320,
-                 "fa_decode_kernel": 160, "fa_decode_merge_kernel": 256,
+                 "fa_fwd_d256_kernel": 352, "fa_decode_kernel": 160, "fa_decode_merge_kernel": 256,
                  "fa_bwd_pre_kernel": 256, "fa_bwd_dq_kernel": 256,
-                 "fa_selftest_wait_kernel": 32}
+                 "fa_selftest_wait_kernel": 32, "fa_selftest_exp2_kernel": 256}
 
 
 def test_every_kernel_fits_the_register_file_at_its_block_size():
@@ -366,3 +370,10 @@ def test_every_kernel_fits_the_register_file_at_its_block_size():
         assert regs * 32 * per_sub <= 16384, (name, res["registers"], BLOCK_THREADS[fam[0]])
         assert res["spill_stores"] <= 8, (name, res)
     assert seen == set(BLOCK_THREADS)
+
+
+def test_selftest_exp2_rejects_bad_arguments(lib):
+    assert lib.fa_selftest_exp2(None, None, 0, None) == fa.FA_OK  # nothing to do, no launch
+    assert lib.fa_selftest_exp2(None, None, -2, None) == fa.FA_ERR_INVALID
+    assert lib.fa_selftest_exp2(None, None, 3, None) == fa.FA_ERR_INVALID
+    assert lib.fa_selftest_exp2(None, None, 4, None) == fa.FA_ERR_INVALID
