@@ -12,6 +12,7 @@
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
+#include "fa_decode_tc.cuh"
 #include "fa_fwd_d256.cuh"
 #include "fa_fwd_pp.cuh"
 
@@ -448,10 +449,45 @@ int launch_decode_nq(const CUtensorMap& k, const CUtensorMap& v, const void* Q,
   return FA_OK;
 }
 
+// The tensor-core form (fa_decode_tc.cuh), d = 128 and kDecTcMinQ..16 rows per head:
+// one CTA per (head, split) whatever the row count.
+template <bool BAND, bool BF16>
+int launch_decode_tc(const CUtensorMap& k, const CUtensorMap& v, const void* Q,
+                     const fa::Strides& sq, void* O, float* L, float* opart, float* lpart, int B,
+                     int H, int Nq, int Nk, const Window& w, fa::TileRange tiles, int splits,
+                     float scale, cudaStream_t stream) {
+  auto kern = fa::fa_decode_tc_kernel<BAND, BF16>;
+  const int smem = static_cast<int>(fa::DtcLayout::kBytes);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  const long BH = static_cast<long>(B) * H;
+  const int tps = tiles.count > 0 ? (tiles.count + splits - 1) / splits : 0;
+  kern<<<static_cast<unsigned>(BH * splits), fa::kDtcThreads, smem, stream>>>(
+      k, v, static_cast<const uint16_t*>(Q), sq, static_cast<uint16_t*>(O), sq, L, opart, lpart,
+      Nq, Nk, H, w.wl, w.wr, tiles.first, tiles.count, tps, splits,
+      scale * 1.4426950408889634074f);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (splits > 1) {
+    const long rows = BH * Nq;
+    fa::fa_decode_merge_kernel<128, BF16><<<static_cast<unsigned>((rows + 7) / 8), 256, 0,
+                                             stream>>>(opart, lpart, static_cast<uint16_t*>(O),
+                                                       sq, L, Nq, H, splits, rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+// Rows per head from which d = 128 decode takes the tensor-core form.
+constexpr int kDecTcMinQ = 2;
+
 template <int D, bool BAND, bool BF16>
 struct DecodeRun {
   template <typename... A>
   static int run(int Nq, A&&... a) {
+    if constexpr (D == 128) {
+      if (Nq >= kDecTcMinQ) return launch_decode_tc<BAND, BF16>(a...);
+    }
     if (Nq <= 1) return launch_decode_nq<D, 1, BAND, BF16>(a...);
     if (Nq <= 4) return launch_decode_nq<D, 4, BAND, BF16>(a...);
     return launch_decode_nq<D, 8, BAND, BF16>(a...);  // 8 rows per CTA
