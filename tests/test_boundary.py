@@ -349,7 +349,7 @@ def test_decode_rejects_before_launch(lib):
 
 # Threads per block of every kernel the library launches.
 BLOCK_THREADS = {"fa_fwd_pp_kernel": 384, "fa_bwd_main_kernel": 512, "fa_bwd_dq_pass_kernel": 320,
-                 "fa_fwd_d256_kernel": 352, "fa_decode_kernel": 160, "fa_decode_merge_kernel": 256,
+                 "fa_fwd_d256_kernel": 352, "fa_decode_kernel": 160, "fa_decode_tc_kernel": 192, "fa_decode_merge_kernel": 256,
                  "fa_bwd_pre_kernel": 256, "fa_bwd_dq_kernel": 256,
                  "fa_selftest_wait_kernel": 32, "fa_selftest_exp2_kernel": 256}
 
