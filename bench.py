@@ -741,7 +741,7 @@ def main():
         extras["by_workload"] = by_w
         hbm = float(peaks["hbm_gbs"])
         extras["decode"] = [time_decode(fa, 4, 32, nq, 65536, 128, dev, stream, 10, 3, hbm)
-                            for nq in (1, 4, 16)]
+                            for nq in (1, 2, 4, 8, 16)]
         extras["latency_small"] = small_call_latency(fa, dev, stream)
         extras["peak_memory"] = peak_memory_vs_n(fa, dev, stream)
         torch.cuda.empty_cache()
