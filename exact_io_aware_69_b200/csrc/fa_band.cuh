@@ -58,4 +58,30 @@ __host__ __device__ inline TileRange query_tiles_of_kv_tile(int j, int tile, int
   return {qlo / tile, qhi / tile - qlo / tile + 1};
 }
 
+// Order of the work items of a launch with a band (whose items differ in cost): block b
+// -> (head bh, rank), rank 0 being each head's heaviest item. Heads go in groups of
+// `group`; within a group the items are rank-major, so that every head's heavy items
+// start early and the launch ends on light ones (no heavy item left to run alone at
+// the end), while the heads in flight at once stay few enough for the tensors they
+// stream to share L2. group = 1 is plain head-major order.
+__host__ __device__ inline void band_order(int b, int per_head, int BH, int group, int* bh,
+                                           int* rank) {
+  const int span = group * per_head;
+  const int g = b / span;
+  const int gg = BH - g * group < group ? BH - g * group : group;  // heads in this group
+  const int idx = b - g * span;
+  *rank = idx / gg;
+  *bh = g * group + (idx - *rank * gg);
+}
+
+// Heads per group for band_order: as many as keep the two streamed 16-bit tensors of
+// the group (2 x n rows x d per head) within 48 MB of the 126 MB L2.
+inline int band_group(long BH, int n, int d) {
+  const long per_head = 4L * n * d;
+  long g = per_head > 0 ? (48L << 20) / per_head : BH;
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return static_cast<int>(g);
+}
+
 }  // namespace fa

@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const float* __restrict__ Dv, float* __restrict__ dq_acc,
                        uint16_t* __restrict__ dK, uint16_t* __restrict__ dV, int Nq, int Nk,
                        int H, int wl, int wr, Strides kv, float scale, float scale_log2,
-                       uint32_t smem_alloc) {
+                       uint32_t smem_alloc, int group) {
   // dS^T for the dK MMA: from TMEM at d = 128, from shared memory at d = 64
   constexpr bool kDsInTmem = D == 128;
   using Lay = BwdLayout<D>;
@@ -221,10 +221,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int lane = threadIdx.x & 31;
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head
   const int ntk = (Nk + kTile - 1) / kTile;  // key tiles per head (one CTA each)
-  const int bh = blockIdx.x / ntk;
+  // band: heads in groups, each group's key tiles rank-major (band_order; under the
+  // causal mask key tile 0 has the most work); otherwise head-major
+  int bh, j;  // j: key tile
+  if (BAND) {
+    band_order(blockIdx.x, ntk, gridDim.x / ntk, group, &bh, &j);
+  } else {
+    bh = blockIdx.x / ntk;
+    j = blockIdx.x - bh * ntk;
+  }
   const int hh = bh % H;  // head
   const int bb = bh / H;  // batch
-  const int j = blockIdx.x - bh * ntk;  // key tile (j = 0 has the most causal work)
   // Rows past Nq / Nk arrive as zeros through the tensor maps. Padded queries, and
   // queries that see no key, have Ls = -inf, so their P is 0. Padded keys of the last
   // key tile need no mask: their dK and dV rows are not stored, and their dS meets

@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                           const __grid_constant__ CUtensorMap tmDO,
                           const __grid_constant__ CUtensorMap tmDQ, const float* __restrict__ Ls,
                           const float* __restrict__ Dv, int Nq, int Nk, int H, int wl, int wr,
-                          float scale, float scale_log2) {
+                          float scale, float scale_log2, int group) {
   using Lay = DqLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -91,10 +91,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   const int lane = threadIdx.x & 31;
   const int ntq = (Nq + kTile - 1) / kTile;
   const int ntk = (Nk + kTile - 1) / kTile;
-  const int bh = blockIdx.x / ntq;
+  // band: heaviest tiles first, heads in groups (band_order); otherwise head-major
+  int bh, tr;
+  if (BAND) {
+    band_order(blockIdx.x, ntq, gridDim.x / ntq, group, &bh, &tr);
+  } else {
+    bh = blockIdx.x / ntq;
+    tr = blockIdx.x - bh * ntq;
+  }
   const int hh = bh % H;
   const int bb = bh / H;
-  const int tr = blockIdx.x - bh * ntq;
   const int t = BAND ? (ntq - 1 - tr) : tr;  // causal: heaviest tiles first
   const TileRange kv = BAND ? kv_tiles_of_query_tile(t, kTile, Nq, Nk, wl, wr)
                             : TileRange{0, ntk};

@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
                        const __grid_constant__ CUtensorMap tmO,
                        const __grid_constant__ CUtensorMap tmOres, bool has_res,
                        float* __restrict__ Lse, int Nq, int Nk, int H, int wl, int wr,
-                       float scale_log2) {
+                       float scale_log2, int group) {
   constexpr int D = kWD;
   using Lay = WideLayout;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -104,10 +104,16 @@ __global__ void __launch_bounds__(kWThreads, 1)
   const int lane = threadIdx.x & 31;
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head (one CTA each)
   const int ntk = (Nk + kTile - 1) / kTile;  // key / value tiles per head
-  const int bh = blockIdx.x / ntq;
+  // band: heaviest tiles first, heads in groups (band_order); otherwise head-major
+  int bh, tr;
+  if (BAND) {
+    band_order(blockIdx.x, ntq, gridDim.x / ntq, group, &bh, &tr);
+  } else {
+    bh = blockIdx.x / ntq;
+    tr = blockIdx.x - bh * ntq;
+  }
   const int hh = bh % H;  // head
   const int bb = bh / H;  // batch
-  const int tr = blockIdx.x - bh * ntq;
   const int t = BAND ? (ntq - 1 - tr) : tr;  // causal: heaviest tiles first
   // The key/value tiles this query tile visits: all of them, or the band's. A tile of
   // only rows that see no key visits none (O = 0, L = -inf).

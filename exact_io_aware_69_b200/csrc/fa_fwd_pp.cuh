@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                      const __grid_constant__ CUtensorMap tmOres, bool has_res,
                      float* __restrict__ Lse, int Nq, int Nk, int H, int wl, int wr,
-                     float scale_log2) {
+                     float scale_log2, int group) {
   using Lay = PpLayout<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -125,10 +125,16 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   const int ntq = (Nq + kTile - 1) / kTile;  // query tiles per head
   const int ntk = (Nk + kTile - 1) / kTile;  // key / value tiles per head
   const int npairs = (ntq + 1) / 2;          // CTAs per head
-  const int bh = blockIdx.x / npairs;
+  // band: heaviest pairs first, heads in groups (band_order); otherwise head-major
+  int bh, pr;
+  if (BAND) {
+    band_order(blockIdx.x, npairs, gridDim.x / npairs, group, &bh, &pr);
+  } else {
+    bh = blockIdx.x / npairs;
+    pr = blockIdx.x - bh * npairs;
+  }
   const int hh = bh % H;
   const int bb = bh / H;
-  const int pr = blockIdx.x - bh * npairs;
   const int pair = BAND ? (npairs - 1 - pr) : pr;  // causal: heaviest pairs first
   // Query tiles 2 pair and 2 pair + 1 (the second may not exist when ntq is odd), and
   // the key tiles each one visits: R_g = [a_g, a_g + n_g).
