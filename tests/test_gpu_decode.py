@@ -61,6 +61,7 @@ CASES = [  # (B, H, Nq, Nk, d, window)
     (1, 2, 7, 6000, 128, (1000, 3)),
     (1, 1, 4, 2, 128, (-1, 0)),          # queries 0 and 1 see no key
     (1, 1, 16, 20000, 128, (10, 0)),     # windows far inside one tile pair
+    (2, 2, 2, 3000, 128, (-1, 0)),       # the fewest rows the tensor-core form takes
 ]
 
 
