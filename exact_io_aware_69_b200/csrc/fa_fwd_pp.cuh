@@ -96,8 +96,9 @@ enum : int {
   kPbVFull = kPbKEmpty + kPpKStages,       // + V stage
   kPbVEmpty = kPbVFull + kPpVStages,       // + V stage
   kPbSFull = kPbVEmpty + kPpVStages,       // + warpgroup
-  kPbPFull = kPbSFull + 2,                 // + warpgroup (128 arrivals)
-  kPbODone = kPbPFull + 2,                 // + warpgroup: its last P V has completed
+  kPbPFull = kPbSFull + 2,                 // + warpgroup (128 arrivals): all of P_g,j
+  kPbPHalf = kPbPFull + 2,                 // + warpgroup (128 arrivals): P_g,j of keys 0-63
+  kPbODone = kPbPHalf + 2,                 // + warpgroup: its last P V has completed
   kPpNumBars = kPbODone + 2,
 };
 static_assert(kPpNumBars <= 20, "barrier area");
@@ -113,6 +114,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                      float* __restrict__ Lse, int Nq, int Nk, int H, int wl, int wr,
                      float scale_log2, int group) {
   using Lay = PpLayout<D>;
+  // P_g,j V_j in two halves at d = 64 (see the MMA issuer)
+  constexpr bool kPpSplitPV = D == 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t pad = ((raw_base + 1023u) & ~1023u) - raw_base;
@@ -179,6 +182,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     for (int g = 0; g < 2; ++g) {
       mbar_init(bar(kPbSFull + g), 1);
       mbar_init(bar(kPbPFull + g), 128);
+      mbar_init(bar(kPbPHalf + g), 128);
       mbar_init(bar(kPbODone + g), 1);
     }
     *abort_flag = 0;
@@ -253,7 +257,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
         for (int g = 0; g < 2; ++g) {
           if (in_range(g, j - 1)) {  // PV_g,j-1: O_g += P_g,j-1 V_j-1
             const int u = j - 1 - first_of(g);  // use count of this warpgroup's buffers
-            if (!mbar_wait(bar(kPbPFull + g), static_cast<uint32_t>(u) & 1, abort_flag)) {
+            // At d = 64 in two halves: keys 0-63 as soon as their P is in TMEM (the
+            // softmax is then still on keys 64-127), keys 64-127 with the rest of P. At
+            // d = 128 (twice the MMA work per key) the split measured no gain.
+            if (!mbar_wait(bar((kPpSplitPV ? kPbPHalf : kPbPFull) + g), static_cast<uint32_t>(u) & 1,
+                           abort_flag)) {
               ok = false;
               break;
             }
@@ -271,9 +279,19 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             const uint32_t a_p = tmem + Lay::tS + g * 128;  // P packed in 64 columns
             const uint32_t d_o = tmem + Lay::tO + g * D;
 #pragma unroll
-            for (int k = 0; k < kTile / 16; ++k)
+            for (int k = 0; k < kTile / 32; ++k)
               mma_ts(d_o, a_p + k * 8, sdesc_step(dv, k * 2048), idesc_o,
                      (u > 0 || k > 0) ? 1u : 0u);
+            if (kPpSplitPV) {
+              if (!mbar_wait(bar(kPbPFull + g), static_cast<uint32_t>(u) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+#pragma unroll
+            for (int k = kTile / 32; k < kTile / 16; ++k)
+              mma_ts(d_o, a_p + k * 8, sdesc_step(dv, k * 2048), idesc_o, 1u);
             if (j == first_of(g) + count_of(g)) mma_commit(bar(kPbODone + g));  // its last P V
             FA_TRACE_EVENT(i, 2 * g);
           }
@@ -370,6 +388,21 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       const float alpha = empty_row ? 1.f : ex2_approx(m - m_new);  // 0 on the first tile
       const float m_sub = empty_row ? 0.f : m_new;
       const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
+      // O_g holds P_g,j-1 V_j-1 already (S_g,j completing implies it); rescale it before
+      // any of P_g,j V_j is issued (the first half goes at the PHalf signal below), only
+      // when a row's reference moved
+      if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_cols + c * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_base + o_cols + c * 32, o);
+        }
+      }
       // packed fp32 pairs, two independent accumulators per sum (16-deep chains)
       uint64_t sum2[2] = {0, 0}, sum2_o[2] = {0, 0};  // packed +0.0f
       // Exponentials on MUFU; on tiles without a mask, kPpPolyPairs of every 16 pairs
@@ -402,6 +435,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           // P packed over the first 64 columns of the S buffer; this thread owns the
           // row, and all of S is in registers already
           tmem_st16(lane_base + s_cols + h * 16, pk);
+          if (kPpSplitPV && h == 1) {  // keys 0-63 (and a rescaled O) in TMEM: their P V may go
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(kPbPHalf + g));
+          }
         }
       };
       if (kPpPolyPairs > 0 && !(hmask || lmask || kmask))
@@ -413,20 +451,6 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       f2_unpack(f2_add(sum2_o[0], sum2_o[1]), b0, b1);
       l = l * alpha + (a0 + a1);
       l_o = l_o * alpha + (b0 + b1);
-      // O_g holds P_g,j-1 V_j-1 already (S_g,j completing implies it); rescale it
-      // before P_g,j V_j is issued, only when a row's reference moved
-      if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + o_cols + c * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_base + o_cols + c * 32, o);
-        }
-      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kPbPFull + g));
