@@ -176,7 +176,9 @@ int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   const unsigned pairs = static_cast<unsigned>(((Nq + fa::kTile - 1) / fa::kTile + 1) / 2);
   const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) * pairs;
   // band: heaviest pairs first within groups of heads that share L2 (K and V streamed)
-  const int group = w.band ? fa::band_group(static_cast<long>(B) * H, Nk, D) : 1;
+  const int group = w.band ? fa::band_group(static_cast<long>(B) * H, 4L * Nk * D,
+                                            fa::kFwdGroupMin, fa::kFwdGroupBytes)
+                           : 1;
   kern<<<grid, fa::kPpThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
                                                 w.wr, scale * 1.4426950408889634074f, group);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -195,7 +197,9 @@ int launch_fwd_d256(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMa
     return FA_ERR_CUDA;
   const unsigned tiles = static_cast<unsigned>((Nq + fa::kTile - 1) / fa::kTile);
   const unsigned grid = static_cast<unsigned>(B) * static_cast<unsigned>(H) * tiles;
-  const int group = w.band ? fa::band_group(static_cast<long>(B) * H, Nk, 256) : 1;
+  const int group = w.band ? fa::band_group(static_cast<long>(B) * H, 4L * Nk * 256,
+                                            fa::kFwdGroupMin, fa::kFwdGroupBytes)
+                           : 1;
   kern<<<grid, fa::kWThreads, smem, stream>>>(q, k, v, o, o_res, has_res, L, Nq, Nk, H, w.wl,
                                               w.wr, scale * 1.4426950408889634074f, group);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -272,7 +276,8 @@ int launch_bwd(const BwdArgs& a, int stages) {
         *a.q, *a.k, *a.v, *a.dO_map, *a.dq_map, Ls, Dv, dq_acc, static_cast<uint16_t*>(a.dK),
         static_cast<uint16_t*>(a.dV), a.Nq, a.Nk, a.H, a.w.wl, a.w.wr, sk, a.scale, scale_log2,
         static_cast<uint32_t>(smem),
-        a.w.band ? fa::band_group(BH, a.Nq, D) : 1);  // Q and dO streamed per key tile
+        // Q and dO streamed per key tile, and the fp32 dQ accumulator added into
+        a.w.band ? fa::band_group(BH, 8L * a.Nq * D, fa::kBwdGroupMin, fa::kBwdGroupBytes) : 1);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if ((stages & FA_STAGE_DQ) && a.det) {
@@ -287,7 +292,10 @@ int launch_bwd(const BwdArgs& a, int stages) {
     kern<<<grid, fa::kDqThreads, smem, a.stream>>>(*a.q, *a.k, *a.v, *a.dO_map, *a.dq_out, Ls,
                                                    Dv, a.Nq, a.Nk, a.H, a.w.wl, a.w.wr, a.scale,
                                                    scale_log2,
-                                                   a.w.band ? fa::band_group(BH, a.Nk, D) : 1);
+                                                   a.w.band ? fa::band_group(BH, 4L * a.Nk * D,
+                                                                             fa::kFwdGroupMin,
+                                                                             fa::kFwdGroupBytes)
+                                                            : 1);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   } else if (stages & FA_STAGE_DQ) {
     const long n8 = rows * D / 8;

@@ -74,14 +74,26 @@ __host__ __device__ inline void band_order(int b, int per_head, int BH, int grou
   *bh = g * group + (idx - *rank * gg);
 }
 
-// Heads per group for band_order: as many as keep the two streamed 16-bit tensors of
-// the group (2 x n rows x d per head) within 48 MB of the 126 MB L2.
-inline int band_group(long BH, int n, int d) {
-  const long per_head = 4L * n * d;
-  long g = per_head > 0 ? (48L << 20) / per_head : BH;
-  if (g < 1) g = 1;
-  if (g > BH) g = BH;
-  return static_cast<int>(g);
+// Heads per group for band_order: at least `min_groups` groups, and more when a group's
+// bytes -- what its heads' work items share through L2: the tensors they stream, and
+// in the backward the fp32 dQ accumulator they add into -- would exceed `budget` bytes
+// of the 126 MB L2; the groups as even as the head count allows. The forward kernels
+// take at least three groups within 96 MB: their heaviest item (a causal head's last
+// query tiles) runs ~12 % of a launch, and with three groups the last group's heaviest
+// items still start early enough to end with it (with more, smaller groups they start
+// near the end and run on alone; with one group all heads' K and V stream at once and
+// overflow L2). The dK/dV kernel, whose heaviest item runs ~5 % of a launch, takes
+// groups within 48 MB.
+inline int band_group(long BH, long bytes_per_head, long min_groups, long budget) {
+  if (BH <= 1) return 1;
+  long ng = (BH * bytes_per_head + budget - 1) / budget;
+  if (ng < min_groups) ng = min_groups;
+  if (ng > BH) ng = BH;
+  return static_cast<int>((BH + ng - 1) / ng);
 }
+constexpr long kFwdGroupMin = 3;
+constexpr long kFwdGroupBytes = 96L << 20;
+constexpr long kBwdGroupMin = 1;
+constexpr long kBwdGroupBytes = 48L << 20;
 
 }  // namespace fa

@@ -37,8 +37,9 @@ GROUP_PROGRAM = r'''
 #define __device__
 #include "fa_band.cuh"
 int main() {
-  long BH; int n, d;
-  while (std::scanf("%ld %d %d", &BH, &n, &d) == 3) std::printf("%d\n", fa::band_group(BH, n, d));
+  long BH, bytes, mg, budget;
+  while (std::scanf("%ld %ld %ld %ld", &BH, &bytes, &mg, &budget) == 4)
+    std::printf("%d\n", fa::band_group(BH, bytes, mg, budget));
   return 0;
 }
 '''
@@ -81,17 +82,25 @@ def test_band_order_is_a_grouped_rank_major_permutation(exes):
             assert items == [(h, r) for h in range(BH) for r in range(per_head)]
 
 
+def _groups(exe, cases):
+    inp = "".join(f"{bh} {b} {mg} {bud}\n" for bh, b, mg, bud in cases)
+    return list(map(int, subprocess.run([exe], input=inp, capture_output=True, text=True,
+                                        check=True).stdout.split()))
+
+
 def test_band_group_sizing(exes):
     _, group = exes
-    cases = [(64, 8192, 128), (16, 65536, 128), (64, 2048, 64), (3, 512, 64), (64, 8192, 256),
-             (1, 1, 64)]
-    inp = "".join(f"{bh} {n} {d}\n" for bh, n, d in cases)
-    out = list(map(int, subprocess.run([group], input=inp, capture_output=True, text=True,
-                                       check=True).stdout.split()))
-    budget = 48 << 20
-    for (bh, n, d), g in zip(cases, out):
+    fwd, bwd = (3, 96 << 20), (1, 48 << 20)
+    cases = [(64, 4 * 8192 * 128, *fwd), (16, 4 * 65536 * 128, *fwd), (64, 4 * 2048 * 64, *fwd),
+             (3, 4 * 512 * 64, *fwd), (64, 8 * 8192 * 128, *bwd), (1, 256, *fwd), (5, 0, *fwd),
+             (2, 1 << 30, *fwd), (16, 8 * 65536 * 128, *bwd)]
+    out = _groups(group, cases)
+    for (bh, per_head, mg, budget), g in zip(cases, out):
         assert 1 <= g <= bh
-        per_head = 4 * n * d
-        assert g == max(1, min(bh, budget // per_head))
-    assert out[0] == 12  # B2 H32 N8192 d128: 4 MB streamed per head
-    assert out[1] == 1   # N = 65536: one head's K and V already take 32 MB
+        ng = min(bh, max(mg, -(-bh * per_head // budget)))
+        assert g == -(-bh // ng), (bh, per_head, g)
+        assert -(-bh // g) >= min(mg, bh)  # at least min_groups groups
+    assert out[0] == 22  # forward, B2 H32 N8192 d128: 3 groups (22, 22 and 20 heads; 88 MB)
+    assert out[1] == 3   # forward, N = 65536: 32 MB of K and V per head
+    assert out[4] == 6   # dK/dV kernel at c3: 8 MB per head with the fp32 dQ accumulator
+    assert out[8] == 1   # dK/dV kernel at N = 65536: one head already takes 64 MB
