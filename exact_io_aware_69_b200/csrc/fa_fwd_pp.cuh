@@ -388,21 +388,25 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       const float alpha = empty_row ? 1.f : ex2_approx(m - m_new);  // 0 on the first tile
       const float m_sub = empty_row ? 0.f : m_new;
       const uint64_t nm2 = f2_pack(-m_sub, -m_sub);
-      // O_g holds P_g,j-1 V_j-1 already (S_g,j completing implies it); rescale it before
-      // any of P_g,j V_j is issued (the first half goes at the PHalf signal below), only
-      // when a row's reference moved
-      if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      // O_g holds P_g,j-1 V_j-1 already (S_g,j completing implies it); it is rescaled,
+      // only when a row's reference moved, before any of P_g,j V_j is issued: ahead of the
+      // exponentials where the first half of P V goes at the PHalf signal, else after
+      // them, where the TMEM round trip no longer delays the P stores
+      auto rescale_o = [&]() {
+        if (u > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + o_cols + c * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + o_cols + c * 32, o);
+            tmem_wait_ld();
+            reg_fence32(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_base + o_cols + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_base + o_cols + c * 32, o);
+          }
         }
-      }
+      };
+      if (kPpSplitPV) rescale_o();
       // packed fp32 pairs, two independent accumulators per sum (16-deep chains)
       uint64_t sum2[2] = {0, 0}, sum2_o[2] = {0, 0};  // packed +0.0f
       // Exponentials on MUFU; on tiles without a mask, kPpPolyPairs of every 16 pairs
@@ -451,6 +455,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       f2_unpack(f2_add(sum2_o[0], sum2_o[1]), b0, b1);
       l = l * alpha + (a0 + a1);
       l_o = l_o * alpha + (b0 + b1);
+      if (!kPpSplitPV) rescale_o();
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kPbPFull + g));
