@@ -77,22 +77,28 @@ __host__ __device__ inline void band_order(int b, int per_head, int BH, int grou
 // Heads per group for band_order: at least `min_groups` groups, and more when a group's
 // bytes -- what its heads' work items share through L2: the tensors they stream, and
 // in the backward the fp32 dQ accumulator they add into -- would exceed `budget` bytes
-// of the 126 MB L2; the groups as even as the head count allows. The forward kernels
-// take at least three groups within 96 MB: their heaviest item (a causal head's last
-// query tiles) runs ~12 % of a launch, and with three groups the last group's heaviest
-// items still start early enough to end with it (with more, smaller groups they start
-// near the end and run on alone; with one group all heads' K and V stream at once and
-// overflow L2). The dK/dV kernel, whose heaviest item runs ~5 % of a launch, takes
-// groups within 48 MB.
+// of the 126 MB L2; the groups as even as the head count allows, and never above the
+// budget. The forward kernels take at least three groups within 88 MiB: their heaviest
+// item (a causal head's last query tiles) runs ~12 % of a launch, and with three groups
+// the last group's heaviest items still start early enough to end with it (with more,
+// smaller groups they start near the end and run on alone); a group of 88 MiB of K and
+// V (22 heads at N = 8192, d = 128) is read from DRAM once, while groups of 96 MiB read
+// it about twice. The dK/dV kernel, whose heaviest item runs ~5 % of a launch, takes
+// groups within 48 MiB.
 inline int band_group(long BH, long bytes_per_head, long min_groups, long budget) {
   if (BH <= 1) return 1;
   long ng = (BH * bytes_per_head + budget - 1) / budget;
   if (ng < min_groups) ng = min_groups;
   if (ng > BH) ng = BH;
-  return static_cast<int>((BH + ng - 1) / ng);
+  long g = (BH + ng - 1) / ng;
+  if (bytes_per_head > 0) {
+    const long cap = budget / bytes_per_head > 1 ? budget / bytes_per_head : 1;
+    if (g > cap) g = cap;
+  }
+  return static_cast<int>(g);
 }
 constexpr long kFwdGroupMin = 3;
-constexpr long kFwdGroupBytes = 96L << 20;
+constexpr long kFwdGroupBytes = 88L << 20;
 constexpr long kBwdGroupMin = 1;
 constexpr long kBwdGroupBytes = 48L << 20;
 

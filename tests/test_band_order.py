@@ -90,17 +90,23 @@ def _groups(exe, cases):
 
 def test_band_group_sizing(exes):
     _, group = exes
-    fwd, bwd = (3, 96 << 20), (1, 48 << 20)
+    fwd, bwd = (3, 88 << 20), (1, 48 << 20)
     cases = [(64, 4 * 8192 * 128, *fwd), (16, 4 * 65536 * 128, *fwd), (64, 4 * 2048 * 64, *fwd),
              (3, 4 * 512 * 64, *fwd), (64, 8 * 8192 * 128, *bwd), (1, 256, *fwd), (5, 0, *fwd),
-             (2, 1 << 30, *fwd), (16, 8 * 65536 * 128, *bwd)]
+             (2, 1 << 30, *fwd), (16, 8 * 65536 * 128, *bwd), (16, 4 * 32768 * 128, *fwd),
+             (16, 4 * 16384 * 128, *fwd), (7, 40 << 20, *fwd)]
     out = _groups(group, cases)
     for (bh, per_head, mg, budget), g in zip(cases, out):
         assert 1 <= g <= bh
         ng = min(bh, max(mg, -(-bh * per_head // budget)))
-        assert g == -(-bh // ng), (bh, per_head, g)
+        cap = max(1, budget // per_head) if per_head else bh
+        assert g == min(-(-bh // ng), cap), (bh, per_head, g)
         assert -(-bh // g) >= min(mg, bh)  # at least min_groups groups
-    assert out[0] == 22  # forward, B2 H32 N8192 d128: 3 groups (22, 22 and 20 heads; 88 MB)
-    assert out[1] == 3   # forward, N = 65536: 32 MB of K and V per head
-    assert out[4] == 6   # dK/dV kernel at c3: 8 MB per head with the fp32 dQ accumulator
-    assert out[8] == 1   # dK/dV kernel at N = 65536: one head already takes 64 MB
+        assert g == 1 or g * per_head <= budget  # a group's bytes stay within the budget
+    assert out[0] == 22  # forward, B2 H32 N8192 d128: 3 groups (22, 22 and 20 heads; 88 MiB)
+    assert out[1] == 2   # forward, N = 65536: 32 MiB of K and V per head (3 would be 96 MiB)
+    assert out[9] == 5   # forward, N = 32768: 16 MiB per head, 5 heads = 80 MiB
+    assert out[10] == 6  # forward, N = 16384: 3 groups of 6 heads, 48 MiB
+    assert out[4] == 6   # dK/dV kernel at c3: 8 MiB per head with the fp32 dQ accumulator
+    assert out[8] == 1   # dK/dV kernel at N = 65536: one head already takes 64 MiB
+    assert out[11] == 2  # 7 heads of 40 MiB: 3 groups would round up to 3 heads (120 MiB)
