@@ -116,14 +116,19 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs. Every
+    sample carries nvidia-smi's timestamp; only those between mark_start() and mark_end()
+    (host times taken right after the synchronizes that open and close the timed region)
+    enter the result, so that the idle moments around the region do not."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, device_index):
         self.proc = None
+        self.window = None
         self.out = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
         self.sel = []
         try:
@@ -143,6 +148,52 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def mark_start(self):
+        self.window = [time.time(), None]
+
+    def mark_end(self):
+        if self.window is not None:
+            self.window[1] = time.time()
+
+    @staticmethod
+    def parse(lines, window=None):
+        """(seconds since the epoch, SM MHz, max SM MHz, active reasons) per sample line,
+        keeping the samples inside `window` = (t0, t1) when one is given."""
+        import datetime
+        out = []
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            t = None
+            for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+                try:
+                    t = datetime.datetime.strptime(parts[0], fmt).timestamp()
+                    break
+                except ValueError:
+                    pass
+            if window is not None and (t is None or not window[0] <= t <= window[1]):
+                continue
+            out.append((t, sm, mx, [n for n, v in zip(ClockSampler.REASONS, parts[5:9])
+                                    if v.lower().startswith("active")]))
+        return out
+
+    @staticmethod
+    def summarise(samples, in_window):
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [x[1] for x in samples]
+        # outside a marked window, the samples under load: the top part of the distribution
+        hi = sm if in_window else [v for v in sm if v >= 0.5 * max(sm)]
+        return {"sm_mhz": statistics.median(hi), "sm_min_mhz": min(hi),
+                "sm_max_mhz": max(x[2] for x in samples),
+                "reasons": sorted({r for x in samples for r in x[3]}), "samples": len(sm),
+                "window": "timed region" if in_window else "whole sampling period"}
+
     def stop(self):
         if self.proc is None:
             return None
@@ -153,28 +204,14 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.out) as fh:
-            for line in fh:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 8:
-                    continue
-                try:
-                    sm.append(float(parts[0]))
-                    mx.append(float(parts[1]))
-                except ValueError:
-                    continue
-                for n, v in zip(names, parts[4:8]):
-                    if v.lower().startswith("active"):
-                        reasons.add(n)
+            lines = fh.readlines()
         os.unlink(self.out)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        # samples under load: the top part of the distribution (idle edges excluded)
-        hi = [s for s in sm if s >= 0.5 * max(sm)]
-        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if self.window is not None and self.window[1] is not None:
+            inside = self.parse(lines, self.window)
+            if inside:
+                return self.summarise(inside, True)
+        return self.summarise(self.parse(lines), False)
 
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -580,11 +617,13 @@ def main():
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
+    sampler.mark_start()
     t_start.record(stream)
     for s in range(args.steps):
         step(events[s])
     t_end.record(stream)
     torch.cuda.synchronize()
+    sampler.mark_end()
     if pg:
         pg.barrier()
     clocks = sampler.stop()
