@@ -66,10 +66,19 @@ constexpr float kPpRescaleSlack = 8.0f;
 #ifndef FA_PP_POLY_PAIRS
 #define FA_PP_POLY_PAIRS 2
 #endif
-constexpr int kPpPolyPairs = FA_PP_POLY_PAIRS;
-static_assert(kPpPolyPairs >= 0 && kPpPolyPairs <= 16 && (kPpPolyPairs & (kPpPolyPairs - 1)) == 0,
-              "poly pairs");
-constexpr int kPpPolyStride = kPpPolyPairs > 0 ? 16 / kPpPolyPairs : 16;
+// At d = 64 (half the MMA work per key tile) its own count: there the polynomial's
+// extra issue slots cost more than the MUFU time it saves (B1 H16 N16384 d64 non-causal
+// on one box, 0 / 2 / 4 / 8 pairs: 1.603 / 1.667 / 1.723 / 1.866 ms), so MUFU only.
+#ifndef FA_PP_POLY_PAIRS_D64
+#define FA_PP_POLY_PAIRS_D64 0
+#endif
+static_assert(FA_PP_POLY_PAIRS >= 0 && FA_PP_POLY_PAIRS <= 16 &&
+                  (FA_PP_POLY_PAIRS & (FA_PP_POLY_PAIRS - 1)) == 0 && FA_PP_POLY_PAIRS_D64 >= 0 &&
+                  FA_PP_POLY_PAIRS_D64 <= 16 && (FA_PP_POLY_PAIRS_D64 & (FA_PP_POLY_PAIRS_D64 - 1)) == 0,
+              "poly pairs: a power of two up to 16, or 0");
+#ifndef FA_PP_RES_IN_K
+#define FA_PP_RES_IN_K 1
+#endif
 constexpr int kPpKStages = 3;
 constexpr int kPpVStages = 2;
 
@@ -114,6 +123,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                      float* __restrict__ Lse, int Nq, int Nk, int H, int wl, int wr,
                      float scale_log2, int group) {
   using Lay = PpLayout<D>;
+  constexpr int kPpPolyPairs = D == 64 ? FA_PP_POLY_PAIRS_D64 : FA_PP_POLY_PAIRS;
+  constexpr int kPpPolyStride = kPpPolyPairs > 0 ? 16 / kPpPolyPairs : 16;
   // P_g,j V_j in two halves at d = 64 (see the MMA issuer)
   constexpr bool kPpSplitPV = D == 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -462,8 +473,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       if (r == 0) FA_TRACE_EVENT(u, 6 + 3 * g);
       m = m_new;
     }
-    // epilogue: O / l_o and O's rounding residual, staged in this warpgroup's Q tile
-    // (free: its last S MMA has completed) and written with TMA stores
+    // epilogue: O / l_o and O's rounding residual, staged in shared memory and written
+    // with TMA stores. O goes to this warpgroup's Q tile (free: its last S MMA has
+    // completed). O_res goes at the same time to the K stage of key tile J1 - 2 + g when
+    // nothing touches that stage any more once this warpgroup's last P V has completed:
+    // warpgroup 1's range must end at J1 (its last P V is then the CTA's last MMA) and
+    // warpgroup 0's at J1 - 1 or J1 (its last P V then follows both S MMAs of tile
+    // J1 - 2); no K load goes past tile J1 - 1. Otherwise O_res follows O through the
+    // Q tile once O has left it.
     ok = __all_sync(0xffffffffu, ok && (gn == 0 || mbar_wait(bar(kPbODone + g), 0, abort_flag)));
     const bool live = t < ntq;
     ok = named_bar_and(gbar, 128, ok) && live;
@@ -471,8 +488,14 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       tc_fence_after();
       const float inv_l = l_o > 0.f ? 1.f / l_o : 0.f;  // rows that see no key: O = 0
       const uint32_t st = sbase + Lay::kQ + g * Lay::kTileBytes;
+      const int res_tile = J1 - 2 + g;
+      const bool res_k = FA_PP_RES_IN_K && has_res && gn > 0 && res_tile >= J0 &&
+                         (g == 1 ? ga + gn == J1 : ga + gn >= J1 - 1);
+      const uint32_t st_res =
+          res_k ? sbase + Lay::kK + static_cast<uint32_t>((res_tile - J0) % kPpKStages) * Lay::kTileBytes
+                : st;
       const int sw = r & 7;
-      uint32_t lw[D / 2];  // O_res, kept until O has left shared memory
+      uint32_t lw[D / 2];  // O_res, kept until O has left shared memory (when st_res = st)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -503,6 +526,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                            st + chunk + static_cast<uint32_t>(((u0 + uu) ^ sw) * 16)),
                        "r"(hw[4 * uu]), "r"(hw[4 * uu + 1]), "r"(hw[4 * uu + 2]), "r"(hw[4 * uu + 3])
                        : "memory");
+        if (res_k) {
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(
+                             st_res + chunk + static_cast<uint32_t>(((u0 + uu) ^ sw) * 16)),
+                         "r"(lw[c * 16 + 4 * uu]), "r"(lw[c * 16 + 4 * uu + 1]),
+                         "r"(lw[c * 16 + 4 * uu + 2]), "r"(lw[c * 16 + 4 * uu + 3])
+                         : "memory");
+        }
       }
       fence_async_smem();
       if (t * kTile + r < Nq)
@@ -513,10 +545,15 @@ __global__ void __launch_bounds__(kPpThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
           tma_store_4d(&tmO, st + c * Lay::kChunkBytes, c * 64, t * kTile, hh, bb);
+        if (res_k) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_store_4d(&tmOres, st_res + c * Lay::kChunkBytes, c * 64, t * kTile, hh, bb);
+        }
         bulk_commit();
-        bulk_wait_read_all();  // the staging tile is read before O_res overwrites it
+        bulk_wait_read_all();  // the staging tiles are read before O_res overwrites O's
       }
-      if (has_res) {
+      if (has_res && !res_k) {
         named_bar_sync(gbar, 128);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
